@@ -1,0 +1,527 @@
+"""Benchmark of the paged-decode hot path on B200; prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pa|reference] [--workload NAME]
+
+A step is one pass of the whole path over one batch of the workload:
+  host block manager (one slot per sequence, copy-on-write pairs, packed block tables)
+  -> pa_copy_blocks (the step's COW pairs) -> pa_cache_write (one new token per sequence)
+  -> pa_decode (plan, split-K decode, log-sum-exp combine).
+`value` is the device-timed throughput of K such steps with every input already in HBM (the
+host-side block management for the step is done before the timed region); `e2e` runs the same
+steps through the Python API from pinned host buffers, with the block manager, the host->device
+copies of the step's inputs and the device->host read of the outputs inside the timed region.
+
+The metric is effective KV bandwidth: the bytes the step must move by definition (every valid
+cached token's K and V once, q, o, block tables, lengths, the new tokens' K/V read and written,
+the COW blocks read and written), divided by the step time.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of the workload
+(sequence-sharded serving, no collective on the data path); value = all ranks' bytes / the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_329_b200 import api  # noqa: E402
+from paged_kv_cache_329_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode-attn effective KV GB/s (% of B200 HBM peak); seqs/s per step"
+
+
+# ---- workload -----------------------------------------------------------------------------------
+
+WORKLOADS = {
+    "gqa8k_bf16": dict(S=256, H=32, Hk=8, d=128, B=16, dtype=torch.bfloat16, lens=lambda: W.gqa8k_lens(256),
+                       desc="GQA bf16 decode at 8k: 256 seqs, 32 q / 8 kv heads, d=128, B=16, context lognormal "
+                            "(median 1024, sigma 1.0) clipped to [16, 8192], shuffled block pool"),
+    "mha13b_fp16": dict(S=64, H=40, Hk=40, d=128, B=16, dtype=torch.float16,
+                        lens=lambda: W.lens_uniform(W.generator(2), 64, 1, 2048),
+                        desc="13B-style MHA fp16: 64 seqs, 40 heads, d=128, B=16, context U[1,2048]"),
+    "long_bf16": dict(S=16, H=64, Hk=8, d=128, B=16, dtype=torch.bfloat16,
+                      lens=lambda: W.lens_uniform(W.generator(5), 16, 16384, 32768),
+                      desc="long-context bf16: 16 seqs, 64 q / 8 kv heads, d=128, B=16, context U[16384,32768]"),
+}
+
+
+class Workload:
+    """Sequences in a native block manager over a shuffled pool, random K/V in HBM."""
+
+    def __init__(self, name, device, seed_offset=0, growth_steps=0):
+        cfg = WORKLOADS[name]
+        self.name, self.cfg = name, cfg
+        self.S, self.H, self.Hk, self.d, self.B, self.dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
+        self.es = torch.finfo(self.dtype).bits // 8
+        lens = cfg["lens"]().tolist()          # context length of each sequence after this step's token
+        B = self.B
+        need = sum(-(-c // B) for c in lens)
+        self.n_blocks = math.ceil(1.25 * need) + self.S * (growth_steps // B + 2)
+        self.mgr = api.BlockManager(self.n_blocks, B)
+        # Shuffle the free stack: take every block, release them in a seeded random order.
+        g = torch.Generator().manual_seed(4242 + seed_offset)
+        blocks = [self.mgr.alloc_block() for _ in range(self.n_blocks)]
+        for i in torch.randperm(self.n_blocks, generator=g).tolist():
+            self.mgr.decref(blocks[i])
+        self.seqs = torch.empty(self.S, dtype=torch.int32)
+        for i, c in enumerate(lens):
+            sid = self.mgr.seq_create()
+            self.mgr.reserve_slots(sid, c - 1)  # tokens cached before this step
+            self.seqs[i] = sid
+        self.max_blocks = max(lens) // B + growth_steps // B + 4
+        self.max_c = max(lens) + growth_steps + 1
+        gen = torch.Generator(device=device).manual_seed(77 + seed_offset)
+        shape = (self.n_blocks, self.Hk, B, self.d)
+        self.k_cache = torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(self.dtype)
+        self.v_cache = torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(self.dtype)
+        self.device = device
+        self.P = api.default_partition(self.S, self.Hk, self.max_c)
+        self.workspace = api.alloc_workspace(self.S, self.H, self.Hk, self.d, self.max_c, self.P, device)
+
+    def host_step(self, slots=None, pairs=None, tables=None, lens=None):
+        """One step of host block management: a slot per sequence, COW pairs, packed tables."""
+        slots, pairs = self.mgr.reserve_slots_batch(self.seqs, 1, slots, pairs)
+        tables, lens = self.mgr.build_block_tables(self.seqs, self.max_blocks, tables, lens)
+        return slots, pairs, tables, lens
+
+    def step_bytes(self, lens, n_pairs):
+        S, H, Hk, d, B, es = self.S, self.H, self.Hk, self.d, self.B, self.es
+        lens = [int(c) for c in lens]
+        kv = sum(lens) * Hk * d * 2 * es
+        decode = kv + S * H * d * es * 2 + 4 * sum(-(-c // B) for c in lens) + 4 * S
+        write = 2 * (S * Hk * d * es * 2) + 8 * S
+        copy = n_pairs * 2 * (Hk * B * d * es) * 2
+        return decode, decode + write + copy, kv
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if its source hash matches."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_gqa8k_bf16.md")
+    src = os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", "pa_decode.cu")
+    try:
+        text = open(path).read()
+        h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text).group(1)
+        t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text).group(1)
+        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        return float(t) if h == cur else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loops run."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.proc = None
+        self.windows = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def finish(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                sm, mx = float(f[1]), float(f[2])
+            except Exception:
+                continue
+            if not any(a - 1.0 <= ts <= b + 1.0 for a, b in self.windows):
+                continue
+            sms.append(sm)
+            maxes.append(mx)
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ---- the GPU arm ----------------------------------------------------------------------------------
+
+def run_pa(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    K, Wm = args.steps, args.warmup
+    e2e_steps = min(K, args.e2e_steps)
+    wl = Workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + 2)
+    S, H, Hk, d = wl.S, wl.H, wl.Hk, wl.d
+    gen = torch.Generator(device=dev).manual_seed(99 + rank)
+    q = torch.randn((S, H, d), generator=gen, device=dev).to(wl.dtype)
+    key = torch.randn((S, Hk, d), generator=gen, device=dev).to(wl.dtype)
+    val = torch.randn((S, Hk, d), generator=gen, device=dev).to(wl.dtype)
+    out = torch.empty((S, H, d), dtype=wl.dtype, device=dev)
+
+    # The step whose inputs sit in HBM for the device-timed loop.
+    slots, pairs, tables, lens = wl.host_step()
+    d_slots, d_pairs = slots.to(dev), pairs.to(dev)
+    d_tables, d_lens = tables.to(dev), lens.to(dev)
+    n_pairs = pairs.shape[0]
+    decode_bytes, step_bytes, kv_bytes = wl.step_bytes(lens.tolist(), n_pairs)
+    max_parts = -(-wl.max_c // wl.P)
+    launches_per_step = 2 + (1 if max_parts > 1 else 0) + 1 + (1 if n_pairs else 0)
+
+    def device_step(ev0=None, ev1=None):
+        if n_pairs:
+            api.pa_copy_blocks(wl.k_cache, wl.v_cache, d_pairs)
+        api.pa_cache_write(wl.k_cache, wl.v_cache, key, val, d_slots)
+        if ev0 is not None:
+            ev0.record()
+        api.pa_decode(q, wl.k_cache, wl.v_cache, d_tables, d_lens, max_context_len=wl.max_c, out=out,
+                      partition_size=wl.P, workspace=wl.workspace)
+        if ev1 is not None:
+            ev1.record()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(local_rank)
+    for _ in range(Wm):
+        device_step()
+    torch.cuda.synchronize()
+    assert api.workspace_error(wl.workspace) == 0, "decode reported an error"
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record()
+    for i in range(K):
+        device_step(*evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    clocks.mark(t_wall0, t_wall1)
+    total_ms = start.elapsed_time(stop)
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    # ---- end to end through the API, from pinned host memory ----
+    pin = lambda t: t.cpu().pin_memory()
+    h_q, h_key, h_val = pin(q), pin(key), pin(val)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_slots = torch.empty(S, dtype=torch.int64).pin_memory()
+    h_pairs = torch.empty((S, 2), dtype=torch.int32).pin_memory()
+    h_tables = torch.empty((S, wl.max_blocks), dtype=torch.int32).pin_memory()
+    h_lens = torch.empty(S, dtype=torch.int32).pin_memory()
+    d_q, d_key, d_val = torch.empty_like(q), torch.empty_like(key), torch.empty_like(val)
+    d_slots2 = torch.empty(S, dtype=torch.int64, device=dev)
+    d_pairs2 = torch.empty((S, 2), dtype=torch.int32, device=dev)
+    d_tables2 = torch.empty((S, wl.max_blocks), dtype=torch.int32, device=dev)
+    d_lens2 = torch.empty(S, dtype=torch.int32, device=dev)
+    e2e_bytes = 0
+    h2d = d2h = 0
+
+    def e2e_step():
+        nonlocal e2e_bytes, h2d, d2h
+        sl, pr, tb, ln = wl.host_step(h_slots, h_pairs, h_tables, h_lens)
+        npairs = pr.shape[0]
+        d_q.copy_(h_q, non_blocking=True)
+        d_key.copy_(h_key, non_blocking=True)
+        d_val.copy_(h_val, non_blocking=True)
+        d_slots2.copy_(sl, non_blocking=True)
+        d_tables2.copy_(tb, non_blocking=True)
+        d_lens2.copy_(ln, non_blocking=True)
+        moved = [h_q, h_key, h_val, sl, tb, ln]
+        if npairs:
+            d_pairs2[:npairs].copy_(pr, non_blocking=True)
+            moved.append(pr)
+            api.pa_copy_blocks(wl.k_cache, wl.v_cache, d_pairs2[:npairs])
+        api.pa_cache_write(wl.k_cache, wl.v_cache, d_key, d_val, d_slots2)
+        api.pa_decode(d_q, wl.k_cache, wl.v_cache, d_tables2, d_lens2, max_context_len=wl.max_c, out=out,
+                      partition_size=wl.P, workspace=wl.workspace)
+        h_out.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        e2e_bytes += wl.step_bytes(ln.tolist(), npairs)[1]
+        h2d += sum(t.numel() * t.element_size() for t in moved)
+        d2h += h_out.numel() * h_out.element_size()
+
+    e2e_step()  # warm-up (also grows every sequence by one token)
+    e2e_bytes = h2d = d2h = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks.mark(t_wall0, time.time())
+    e2e_ms = e0.elapsed_time(e1)
+    clock_info = clocks.finish()
+
+    # max over ranks
+    t = torch.tensor([total_ms, e2e_ms, decode_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms, decode_ms = t.tolist()
+    if rank != 0:
+        return None
+
+    peak, peak_kind = load_peaks()
+    value = world * step_bytes * K / (total_ms * 1e-3) / 1e9
+    achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
+    ms_per_step = total_ms / K
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[wl.dtype],
+        "data": "synthetic",
+        "config": {
+            "workload": wl.cfg["desc"],
+            "global_batch": S * world,
+            "seq_len": f"mean {statistics.mean(lens.tolist()):.0f}, max {max(lens.tolist())}",
+            "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
+            "partition_size": wl.P,
+            "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush",
+            "step": "host block manager -> pa_copy_blocks -> pa_cache_write -> pa_decode (plan, decode, combine)",
+            "step_bytes": step_bytes,
+            "cow_pairs_per_step": n_pairs,
+        },
+        "seqs_per_s": round(S * world / (ms_per_step * 1e-3), 1),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "pa_decode (plan + decode_kernel + combine, CUDA events around the call)",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(),
+            "algorithmic_bytes_per_launch": decode_bytes,
+            "launch_ms": round(decode_ms, 5),
+        },
+        "clocks": clock_info,
+        "e2e": {
+            "value": round(world * e2e_bytes / (e2e_ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": h2d // max(e2e_steps, 1),
+            "d2h_bytes_per_step": d2h // max(e2e_steps, 1),
+            "steps": e2e_steps,
+            "ms_per_step": round(e2e_ms / e2e_steps, 5),
+            "note": "host block manager + H2D of the step's inputs + kernels + D2H of o, synchronised each step",
+        },
+        "gpu_launches": K * launches_per_step,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, lens.tolist(), q, target_s=args.cpu_seconds)
+    return line
+
+
+# ---- the oracle on the host cores -----------------------------------------------------------------
+
+def _compact(wl, sample, q_dev=None, tables=None, lens=None, device_cache=True):
+    """CPU copies of the sampled sequences' blocks, with a remapped table."""
+    t = tables[sample]
+    used = torch.unique(t[t >= 0])
+    remap = torch.full((wl.n_blocks,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(used.numel(), dtype=torch.int32)
+    t2 = torch.where(t >= 0, remap[t.clamp(min=0).long()], t)
+    kc = wl.k_cache[used.to(wl.k_cache.device)].cpu()
+    vc = wl.v_cache[used.to(wl.v_cache.device)].cpu()
+    return q_dev[sample].cpu(), kc, vc, t2, lens[sample]
+
+
+def cpu_baseline(wl, lens, q, target_s=12.0):
+    import oracle
+
+    oracle.build()
+    tables, lens_t = wl.mgr.build_block_tables(wl.seqs, wl.max_blocks)
+    cores = oracle.hardware_threads()
+    order = torch.randperm(wl.S, generator=torch.Generator().manual_seed(5)).tolist()
+    # calibrate on two sequences, then size the sample for ~target_s seconds
+    probe = order[:2]
+    qs, kc, vc, t2, ls = _compact(wl, torch.tensor(probe), q, tables, lens_t)
+    t0 = time.perf_counter()
+    oracle.decode(qs, kc, vc, t2, ls, n_threads=0)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    per_tok = dt / max(1, int(ls.sum()))
+    n_tok_target = target_s / per_tok
+    sample, acc = [], 0
+    for s in order:
+        if acc >= n_tok_target:
+            break
+        sample.append(s)
+        acc += int(lens_t[s])
+    qs, kc, vc, t2, ls = _compact(wl, torch.tensor(sample), q, tables, lens_t)
+    t0 = time.perf_counter()
+    oracle.decode(qs, kc, vc, t2, ls, n_threads=0)
+    dt = time.perf_counter() - t0
+    es, Hk, d, H, B = wl.es, wl.Hk, wl.d, wl.H, wl.B
+    c = [int(x) for x in ls]
+    byt = sum(c) * Hk * d * 2 * es + len(c) * H * d * es * 2 + 4 * sum(-(-x // B) for x in c) + 4 * len(c)
+    return {"value": round(byt / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} of {wl.S} sequences ({sum(c)} tokens x {H} heads), decode only, "
+                      f"fp64 C++ oracle with {cores} threads, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores, one bounded sample of the workload per step."""
+    if rank != 0:
+        return None
+    import oracle
+
+    oracle.build()
+    cfg = WORKLOADS[args.workload]
+    lens = cfg["lens"]().tolist()
+    S, H, Hk, d, B, dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
+    es = torch.finfo(dtype).bits // 8
+    cores = oracle.hardware_threads()
+    # Per-step sample: a slice of sequences, generated on the CPU with the workload's shapes.
+    budget = 100.0 / (args.steps + args.warmup)       # seconds of oracle work per step
+    g = torch.Generator().manual_seed(6)
+
+    def make(seqs):
+        ls = [lens[s] for s in seqs]
+        case = W.paged_case("ref", ls, H, Hk, d, B, dtype, 1234 + seqs[0], sentinel="none", pool_factor=1.0)
+        return case
+
+    probe = make([0])
+    t0 = time.perf_counter()
+    oracle.decode(probe.q, probe.k_cache, probe.v_cache, probe.block_tables, probe.context_lens, n_threads=0)
+    per_tok = (time.perf_counter() - t0) / lens[0]
+    tok_budget = max(16, int(budget / per_tok))
+    # rotate through the sequences; a sequence longer than the budget is cut to the budget
+    cases, s = [], 0
+    for i in range(min(args.steps + args.warmup, 64)):
+        ls = min(lens[s % S], tok_budget)
+        case = W.paged_case("ref", [ls], H, Hk, d, B, dtype, 1234 + i, sentinel="none", pool_factor=1.0)
+        cases.append(case)
+        s += 1
+    times, bytes_ = [], []
+    for i in range(args.warmup + args.steps):
+        c = cases[i % len(cases)]
+        t0 = time.perf_counter()
+        oracle.decode(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, n_threads=0)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            n = int(c.context_lens.sum())
+            bytes_.append(n * Hk * d * 2 * es + c.S * H * d * es * 2 + 4 * (-(-n // B)) + 4 * c.S)
+    total = sum(times)
+    value = sum(bytes_) / total / 1e9
+    sample = (f"each step: one sequence of the workload (cut to <= {tok_budget} tokens), {H} heads, decode only; "
+              f"fp64 C++ oracle, {cores} threads")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg["desc"], "global_batch": S, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
+    ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        backend = "nccl" if args.impl == "pa" else "gloo"
+        if args.impl == "pa":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            from paged_kv_cache_329_b200 import build
+
+            if rank == 0 and not os.path.exists(os.path.join(ROOT, "paged_kv_cache_329_b200", "libpa.so")):
+                build.build()
+            if world > 1:
+                torch.distributed.barrier()
+            line = run_pa(args, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

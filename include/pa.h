@@ -1,0 +1,233 @@
+/*
+ * pa.h -- C ABI of libpa: paged decode attention on NVIDIA B200 (sm_100a).
+ *
+ * The library computes the decode step of attention over a KV cache that is stored in fixed-size
+ * physical blocks, and carries the two data-parallel paths that keep such a cache up to date
+ * (the slot-mapped write of new tokens and the copy-on-write block copy), plus a host-side block
+ * manager with reference counts that produces the block tables, slot mappings and copy pairs.
+ *
+ * Sources (page title, section, equation or list):
+ *   "PagedAttention原理" (scmmm.top), "为什么会有 KV cache": o_t = softmax(q_t K^T / sqrt(d)) V
+ *   "PagedAttention原理", "实现一个虚拟内存": K_j = (k_{(j-1)B+1} .. k_{jB}), V_j likewise,
+ *       A_ij = exp(q_i^T K_j / sqrt(d)) / sum_t exp(q_i^T K_t / sqrt(d)),  o_i = sum_j V_j A_ij^T;
+ *       the block table records, per logical block, its physical block and its fill count.
+ *   "PagedAttention原理", "从虚拟内存的启发": blocks of B tokens requested one at a time.
+ *   "PagedAttention原理", "解决共享prompt" and "解决COW": per-block reference counts and the five
+ *       copy-on-write steps; "COW 区别": a block with free slots is appended to without copying.
+ *   "vllm" (cnblogs), section 2.2 Decode: each decode step appends the new token's K and V.
+ *
+ * Conventions for every entry point below.
+ *   - Tensors are dense, row-major, contiguous.  "device" pointers point to memory the caller
+ *     allocated on the current CUDA device; "host" pointers to host memory.  The library never
+ *     takes ownership of a caller's buffer and never allocates device memory.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Device work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *     runs asynchronously: a return of PA_OK means the arguments were valid and the kernels were
+ *     launched.  Faults inside a kernel surface at the caller's next synchronisation.
+ *   - No C++ exception crosses this boundary.  On failure an entry point returns a pa_status
+ *     other than PA_OK and pa_last_error() returns a message (per host thread).
+ *   - Shapes: S sequences, H query heads, Hk kv heads (H % Hk == 0; query head h reads kv head
+ *     h / (H / Hk)), head dimension d, block size B (tokens per block), n_blocks physical blocks.
+ *   - Supported: d in {64, 128}; B in {8, 16, 32}; H / Hk in {1, 2, 4, 8}; element types
+ *     PA_F32, PA_F16, PA_BF16 (query and caches share one type).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* bad shape, type, pointer, alignment or size */
+  PA_ERR_NO_FREE_BLOCK = 2, /* block pool exhausted; the call changed nothing */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_UNSUPPORTED = 4    /* valid request outside the supported set above */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Message for the last failure on the calling host thread ("" if none).  The string is owned by
+ * the library and stays valid until the thread's next call into it. */
+const char* pa_last_error(void);
+
+/* Library version string, static storage. */
+const char* pa_version(void);
+
+/* ---------------------------------------------------------------------------------------------
+ * Paged decode attention.
+ *
+ * For every sequence s (context length c = context_lens[s], which counts the token written in
+ * this step) and query head h with kv head kh = h / (H / Hk):
+ *     x_t = scale * <query[s][h], k_t>          for t = 0 .. c-1,
+ *     out[s][h] = sum_t softmax(x)_t * v_t,
+ * where k_t = k_cache[block_tables[s][t / B]][kh][t % B] and v_t likewise ("实现一个虚拟内存",
+ * eqs. A_ij, o_i; "为什么会有 KV cache", eq. o_t).  Only the c valid tokens are read: slots past
+ * c in the last block and table entries past ceil(c / B) are never used.  c = 0 gives zeros.
+ * Scores, the softmax and the weighted sum are computed in fp32.
+ *
+ * The context is cut into partitions of `partition_size` tokens (a multiple of 64; 0 = chosen by
+ * the library from S, Hk and max_context_len).  Each (sequence, kv head, partition) is one unit of
+ * work; partitions of one sequence are merged by the log-sum-exp combine (pa_combine's rule).
+ * For a fixed partition size the result is a deterministic function of the logical contents:
+ * repeating a call, or moving blocks to other physical ids and updating the table, gives
+ * bit-identical output.
+ *
+ *   out            device, [S][H][d] of out_dtype (any of the three types)
+ *   query          device, [S][H][d] of kv_dtype
+ *   k_cache        device, [n_blocks][Hk][B][d] of kv_dtype
+ *   v_cache        device, [n_blocks][Hk][B][d] of kv_dtype
+ *   block_tables   device, [S][max_blocks_per_seq] int32 physical block ids
+ *   context_lens   device, [S] int32, each in [0, max_context_len]
+ *   max_context_len  host bound on every context_lens[s] (sizes the partition grid)
+ *   scale          score scale, normally 1/sqrt(d)
+ *   workspace      device scratch of at least pa_decode_workspace_size(...) bytes, 256-byte
+ *                  aligned, owned by the caller; its contents need no initialisation and are
+ *                  overwritten.  Calls that overlap on the GPU must not share a workspace.
+ * A block-table entry outside [0, n_blocks) reads as zeros and sets the error word read by
+ * pa_workspace_error().
+ */
+size_t pa_decode_workspace_size(int S, int H, int Hk, int d, int max_context_len, int partition_size);
+
+pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                    int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq,
+                    int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Partition size (tokens) that pa_decode uses for these arguments when given 0. */
+int pa_decode_default_partition(int S, int Hk, int max_context_len);
+
+/* Copies the error word of a decode workspace to *flags (host) after synchronising `stream`.
+ * 0 = no error; bit 0 = a block-table entry was out of range (read as zeros); bit 1 = a pipeline
+ * wait timed out (the kernel gave up); bit 2 = a context length exceeded max_context_len (cut to it). */
+pa_status pa_workspace_error(const void* workspace, int* flags, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Log-sum-exp merge of per-partition partial states ("实现一个虚拟内存", eq. A_ij: its denominator
+ * is a sum over blocks, so it can be accumulated over any partition of the blocks and merged).
+ *
+ * Partition p of sequence s covers tokens [p*P, min((p+1)*P, c)), with P = partition_size and
+ * n_parts(s) = ceil(c / P) (c = context_lens[s]).  For each (s, h) and p < n_parts(s):
+ *   part_m[s][h][p]  = max score m_p over the partition (natural-log units, scores scale*q.k)
+ *   part_l[s][h][p]  = sum over the partition of exp(x_t - m_p)
+ *   part_o[s][h][p]  = sum over the partition of exp(x_t - m_p) * v_t        (d floats)
+ * and the output is  out[s][h] = sum_p w_p part_o_p / sum_p w_p part_l_p,  w_p = exp(m_p - max m).
+ * Entries with p >= n_parts(s) are not read.  c = 0 gives zeros.
+ *
+ *   out      device [S][H][d] of out_dtype
+ *   part_o   device [S][H][max_parts][d] float32
+ *   part_m   device [S][H][max_parts] float32
+ *   part_l   device [S][H][max_parts] float32
+ *   context_lens  device [S] int32, ceil(c / P) <= max_parts
+ */
+pa_status pa_combine(void* out, pa_dtype out_dtype, const float* part_o, const float* part_m,
+                     const float* part_l, const int32_t* context_lens, int S, int H, int d,
+                     int max_parts, int partition_size, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Slot-mapped cache write ("vllm" 2.2 Decode: after each step the new token's K,V go into the
+ * cache; "实现一个虚拟内存": a token's place is its block and its offset in the block).
+ * For every token n with slot = slot_mapping[n] >= 0 and every kv head kh:
+ *     k_cache[slot / B][kh][slot % B][:] = key[n][kh][:],   v_cache likewise from value.
+ * slot < 0 marks a padding token and writes nothing.  Copies are bit-exact.  Two tokens with the
+ * same slot race (the result is one of them).  slot / B must be < n_blocks: out-of-range slots are
+ * skipped on the device and reported by nothing else, so validate slot mappings on the host when
+ * they do not come from the block manager below.
+ *
+ *   k_cache, v_cache  device [n_blocks][Hk][B][d] of dtype
+ *   key, value        device [T][Hk][d] of dtype
+ *   slot_mapping      device [T] int64
+ */
+pa_status pa_cache_write(void* k_cache, void* v_cache, const void* key, const void* value,
+                         const int64_t* slot_mapping, int T, int Hk, int d, int B, int n_blocks,
+                         pa_dtype dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Copy-on-write block copy ("解决COW", step 2: copy the shared block's contents into the new
+ * block).  For each pair p: block pairs[p][1] of k_cache and of v_cache becomes a bit copy of
+ * block pairs[p][0] (all Hk heads, all B slots).  Destinations must be distinct and no
+ * destination may also be a source in the same call (the block manager's pairs satisfy this);
+ * otherwise the result is undefined.  Out-of-range ids are skipped on the device.
+ *
+ *   pairs   device [P][2] int32 (src, dst)
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int P, int Hk, int d,
+                         int B, int n_blocks, pa_dtype dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Host block manager ("从虚拟内存的启发", "解决共享prompt", "解决COW", "COW 区别").  Pure CPU; a handle
+ * must not be used by two threads at once.  Policies (the pages leave them open):
+ *   - free blocks form a LIFO stack that starts as [n_blocks-1, ..., 1, 0]: the first allocation
+ *     returns 0 and the most recently freed block is handed out next;
+ *   - sequence ids are 0, 1, 2, ... in creation order and are never reused;
+ *   - freeing a sequence releases its blocks in logical order;
+ *   - a reservation that cannot get every block it needs fails with PA_ERR_NO_FREE_BLOCK and
+ *     leaves all state unchanged.
+ */
+typedef struct pa_alloc pa_alloc;
+
+/* New manager over n_blocks physical blocks of B tokens; NULL on bad arguments. */
+pa_alloc* pa_alloc_create(int n_blocks, int B);
+void pa_alloc_destroy(pa_alloc* a);
+
+/* Take one free block with reference count 1. */
+pa_status pa_alloc_block(pa_alloc* a, int32_t* block_id);
+/* Reference counting of an allocated block; decref releases the block when the count hits 0. */
+pa_status pa_block_incref(pa_alloc* a, int32_t block_id);
+pa_status pa_block_decref(pa_alloc* a, int32_t block_id);
+/* Current count (0 = free), or -1 for an id out of range. */
+int pa_block_refcount(const pa_alloc* a, int32_t block_id);
+int pa_alloc_num_free(const pa_alloc* a);
+
+/* Sequences: an empty sequence; a fork that shares every block of the parent (each block's count
+ * goes up by one; the child has the parent's length); free (every block's count goes down by
+ * one).  Parallel sampling and beam search build on fork ("Paged Attention&Orca Paper笔记与解读",
+ * parallel sampling and beam search items). */
+pa_status pa_seq_create(pa_alloc* a, int32_t* seq_id);
+pa_status pa_seq_fork(pa_alloc* a, int32_t parent, int32_t* child);
+pa_status pa_seq_free(pa_alloc* a, int32_t seq_id);
+/* Length (tokens) of a sequence, or -1 if unknown. */
+int pa_seq_len(const pa_alloc* a, int32_t seq_id);
+
+/* Reserve the slots of the next n_new tokens of a sequence.
+ * For each new token, in order:
+ *   - the last block is full (or there is none): take a fresh block; nothing is copied, even if
+ *     the full block is shared;
+ *   - the last block has room and count 1: write in place;
+ *   - the last block has room and count > 1: copy-on-write -- (1) take a new block, (2) emit the
+ *     pair (old, new) for pa_copy_blocks, (3) map the logical block to the new block,
+ *     (4) decrement the old block's count, (5) the token's slot is in the new block.
+ * slots      host [n_new] int64: slot = physical_block * B + offset, for pa_cache_write.
+ * cow_pairs  host [>= 1][2] int32 (src, dst), filled with *n_cow pairs (0 or 1 per call).
+ * The caller copies first (pa_copy_blocks), then writes (pa_cache_write), then decodes. */
+pa_status pa_seq_reserve_slots(pa_alloc* a, int32_t seq_id, int n_new, int64_t* slots,
+                               int32_t* cow_pairs, int* n_cow);
+
+/* One decode step of a batch: reserves n_new slots for each of seq_ids[0..S), in order, exactly as
+ * S calls of pa_seq_reserve_slots would.  slots: host [S * n_new] int64 (sequence i's slots at
+ * i*n_new).  cow_pairs: host [S][2] int32, filled with *n_cow pairs.  Each sequence's reservation
+ * is atomic; on the first failure the call stops, sets *n_done to the number of sequences already
+ * reserved (their slots and pairs are valid) and returns that failure's status.  On success
+ * *n_done = S. */
+pa_status pa_seq_reserve_slots_batch(pa_alloc* a, const int32_t* seq_ids, int S, int n_new, int64_t* slots,
+                                     int32_t* cow_pairs, int* n_cow, int* n_done);
+
+/* Number of blocks in a sequence's table, or -1 if unknown. */
+int pa_seq_num_blocks(const pa_alloc* a, int32_t seq_id);
+
+/* Pack the block tables of seq_ids[0..S) into host tables [S][max_blocks_per_seq] (unused entries
+ * -1) and their lengths into host context_lens [S].  PA_ERR_INVALID_ARG if a sequence is unknown
+ * or has more than max_blocks_per_seq blocks (nothing is written then). */
+pa_status pa_build_block_tables(const pa_alloc* a, const int32_t* seq_ids, int S, int32_t* tables,
+                                int max_blocks_per_seq, int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

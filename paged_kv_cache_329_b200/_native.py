@@ -1,0 +1,66 @@
+"""ctypes loader for libpa.so: declares every C entry point of include/pa.h.
+
+The library is built in-tree (``python -m paged_kv_cache_329_b200.build``).  There is no fallback:
+if libpa.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+F = ctypes.c_float
+SZ = ctypes.c_size_t
+I32P = ctypes.POINTER(ctypes.c_int32)
+I64P = ctypes.POINTER(ctypes.c_int64)
+IP = ctypes.POINTER(ctypes.c_int)
+
+# name -> (restype, argtypes); mirrors include/pa.h
+SIGNATURES = {
+    "pa_last_error": (ctypes.c_char_p, []),
+    "pa_version": (ctypes.c_char_p, []),
+    "pa_decode_workspace_size": (SZ, [I, I, I, I, I, I]),
+    "pa_decode": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
+    "pa_decode_default_partition": (I, [I, I, I]),
+    "pa_workspace_error": (I, [P, IP, P]),
+    "pa_combine": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),
+    "pa_cache_write": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
+    "pa_copy_blocks": (I, [P, P, P, I, I, I, I, I, I, P]),
+    "pa_alloc_create": (P, [I, I]),
+    "pa_alloc_destroy": (None, [P]),
+    "pa_alloc_block": (I, [P, I32P]),
+    "pa_block_incref": (I, [P, ctypes.c_int32]),
+    "pa_block_decref": (I, [P, ctypes.c_int32]),
+    "pa_block_refcount": (I, [P, ctypes.c_int32]),
+    "pa_alloc_num_free": (I, [P]),
+    "pa_seq_create": (I, [P, I32P]),
+    "pa_seq_fork": (I, [P, ctypes.c_int32, I32P]),
+    "pa_seq_free": (I, [P, ctypes.c_int32]),
+    "pa_seq_len": (I, [P, ctypes.c_int32]),
+    "pa_seq_num_blocks": (I, [P, ctypes.c_int32]),
+    "pa_seq_reserve_slots": (I, [P, ctypes.c_int32, I, I64P, I32P, IP]),
+    "pa_seq_reserve_slots_batch": (I, [P, I32P, I, I, I64P, I32P, IP, IP]),
+    "pa_build_block_tables": (I, [P, I32P, I, I32P, I, I32P]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libpa.so not found at {LIB_PATH}; build it with `python -m paged_kv_cache_329_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib

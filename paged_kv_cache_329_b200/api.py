@@ -1,0 +1,226 @@
+"""Python binding of libpa: argument marshalling only; every step runs in the C/CUDA library.
+
+torch supplies device memory and the current CUDA stream.  Each function here checks tensor
+placement and types, then calls the C entry point of the same name (include/pa.h) and raises
+``PAError`` on a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _native
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_NO_FREE_BLOCK, PA_ERR_CUDA, PA_ERR_UNSUPPORTED = range(5)
+DTYPE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"[pa status {status}] {msg}")
+        self.status = status
+
+
+class NoFreeBlock(PAError):
+    pass
+
+
+def _check(status: int):
+    if status != PA_OK:
+        msg = _native.load().pa_last_error().decode(errors="replace")
+        raise (NoFreeBlock if status == PA_ERR_NO_FREE_BLOCK else PAError)(status, msg)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("expected contiguous CUDA tensors")
+
+
+def version() -> str:
+    return _native.load().pa_version().decode()
+
+
+# ---- decode -------------------------------------------------------------------------------------
+
+def default_partition(S: int, Hk: int, max_context_len: int) -> int:
+    return _native.load().pa_decode_default_partition(S, Hk, max_context_len)
+
+
+def decode_workspace_size(S, H, Hk, d, max_context_len, partition_size=0) -> int:
+    return _native.load().pa_decode_workspace_size(S, H, Hk, d, max_context_len, partition_size)
+
+
+def alloc_workspace(S, H, Hk, d, max_context_len, partition_size=0, device="cuda") -> torch.Tensor:
+    n = decode_workspace_size(S, H, Hk, d, max_context_len, partition_size)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, context_lens, *, max_context_len, scale=None, out=None,
+              out_dtype=None, partition_size=0, workspace=None, stream=None):
+    """Paged decode attention; returns out [S, H, d].  See pa_decode in include/pa.h."""
+    _cuda(q, k_cache, v_cache, block_tables, context_lens)
+    S, H, d = q.shape
+    n_blocks, Hk, B, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape or q.dtype != k_cache.dtype or v_cache.dtype != k_cache.dtype:
+        raise ValueError("shape/dtype mismatch between q and the caches")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables and context_lens must be int32")
+    if out is None:
+        out = torch.empty((S, H, d), dtype=out_dtype or q.dtype, device=q.device)
+    _cuda(out)
+    if workspace is None:
+        workspace = alloc_workspace(S, H, Hk, d, max_context_len, partition_size, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(_native.load().pa_decode(
+        _ptr(out), DTYPE[out.dtype], _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), S, H, Hk, d, B, n_blocks, block_tables.shape[1], int(max_context_len),
+        float(scale), DTYPE[q.dtype], int(partition_size), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out
+
+
+def workspace_error(workspace, stream=None) -> int:
+    flags = ctypes.c_int(0)
+    _check(_native.load().pa_workspace_error(_ptr(workspace), ctypes.byref(flags), _stream(stream)))
+    return flags.value
+
+
+def pa_combine(part_o, part_m, part_l, context_lens, partition_size, *, out=None, out_dtype=torch.float32,
+               stream=None):
+    """Log-sum-exp merge of per-partition states; see pa_combine in include/pa.h."""
+    _cuda(part_o, part_m, part_l, context_lens)
+    S, H, max_parts, d = part_o.shape
+    if out is None:
+        out = torch.empty((S, H, d), dtype=out_dtype, device=part_o.device)
+    _check(_native.load().pa_combine(
+        _ptr(out), DTYPE[out.dtype], _ptr(part_o), _ptr(part_m), _ptr(part_l), _ptr(context_lens),
+        S, H, d, max_parts, int(partition_size), _stream(stream)))
+    return out
+
+
+# ---- cache maintenance --------------------------------------------------------------------------
+
+def pa_cache_write(k_cache, v_cache, key, value, slot_mapping, stream=None):
+    _cuda(k_cache, v_cache, key, value, slot_mapping)
+    n_blocks, Hk, B, d = k_cache.shape
+    if slot_mapping.dtype != torch.int64 or key.dtype != k_cache.dtype or value.dtype != k_cache.dtype:
+        raise ValueError("slot_mapping must be int64 and key/value must match the cache type")
+    _check(_native.load().pa_cache_write(
+        _ptr(k_cache), _ptr(v_cache), _ptr(key), _ptr(value), _ptr(slot_mapping), key.shape[0], Hk, d, B,
+        n_blocks, DTYPE[k_cache.dtype], _stream(stream)))
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
+    _cuda(k_cache, v_cache, pairs)
+    n_blocks, Hk, B, d = k_cache.shape
+    if pairs.dtype != torch.int32:
+        raise ValueError("pairs must be int32 [P, 2]")
+    _check(_native.load().pa_copy_blocks(
+        _ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.numel() // 2, Hk, d, B, n_blocks,
+        DTYPE[k_cache.dtype], _stream(stream)))
+
+
+# ---- host block manager -------------------------------------------------------------------------
+
+class BlockManager:
+    """Reference-counted block pool with sequences (pa_alloc_* / pa_seq_* in include/pa.h)."""
+
+    def __init__(self, n_blocks: int, block_size: int):
+        self._lib = _native.load()
+        self._h = self._lib.pa_alloc_create(n_blocks, block_size)
+        if not self._h:
+            raise PAError(PA_ERR_INVALID_ARG, self._lib.pa_last_error().decode())
+        self.n_blocks = n_blocks
+        self.B = block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            self._lib.pa_alloc_destroy(h)
+            self._h = None
+
+    def alloc_block(self) -> int:
+        b = ctypes.c_int32()
+        _check(self._lib.pa_alloc_block(self._h, ctypes.byref(b)))
+        return b.value
+
+    def incref(self, b: int):
+        _check(self._lib.pa_block_incref(self._h, b))
+
+    def decref(self, b: int):
+        _check(self._lib.pa_block_decref(self._h, b))
+
+    def refcount(self, b: int) -> int:
+        return self._lib.pa_block_refcount(self._h, b)
+
+    def num_free(self) -> int:
+        return self._lib.pa_alloc_num_free(self._h)
+
+    def seq_create(self) -> int:
+        s = ctypes.c_int32()
+        _check(self._lib.pa_seq_create(self._h, ctypes.byref(s)))
+        return s.value
+
+    def seq_fork(self, parent: int) -> int:
+        s = ctypes.c_int32()
+        _check(self._lib.pa_seq_fork(self._h, parent, ctypes.byref(s)))
+        return s.value
+
+    def seq_free(self, sid: int):
+        _check(self._lib.pa_seq_free(self._h, sid))
+
+    def seq_len(self, sid: int) -> int:
+        return self._lib.pa_seq_len(self._h, sid)
+
+    def seq_num_blocks(self, sid: int) -> int:
+        return self._lib.pa_seq_num_blocks(self._h, sid)
+
+    def reserve_slots(self, sid: int, n_new: int):
+        """Returns (slots: list[int], cow_pairs: list[(src, dst)])."""
+        slots = (ctypes.c_int64 * max(n_new, 1))()
+        pairs = (ctypes.c_int32 * 2)()
+        n_cow = ctypes.c_int(0)
+        _check(self._lib.pa_seq_reserve_slots(self._h, sid, n_new, slots, pairs, ctypes.byref(n_cow)))
+        return list(slots[:n_new]), [(pairs[2 * i], pairs[2 * i + 1]) for i in range(n_cow.value)]
+
+    def reserve_slots_batch(self, seq_ids, n_new: int = 1, slots=None, pairs=None):
+        """One step for a batch: n_new slots per sequence.  Returns (slots int64 [S*n_new] tensor,
+        pairs int32 [n_cow, 2] tensor).  `slots`/`pairs` may be preallocated (pinned) CPU tensors."""
+        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
+        S = ids.numel()
+        if slots is None:
+            slots = torch.empty(S * n_new, dtype=torch.int64)
+        if pairs is None:
+            pairs = torch.empty((max(S, 1), 2), dtype=torch.int32)
+        n_cow, n_done = ctypes.c_int(0), ctypes.c_int(0)
+        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+        i64 = ctypes.cast(slots.data_ptr(), ctypes.POINTER(ctypes.c_int64))
+        _check(self._lib.pa_seq_reserve_slots_batch(self._h, i32(ids), S, n_new, i64, i32(pairs),
+                                                    ctypes.byref(n_cow), ctypes.byref(n_done)))
+        return slots, pairs[: n_cow.value]
+
+    def build_block_tables(self, seq_ids, max_blocks_per_seq: int, tables=None, lens=None):
+        """Returns (tables int32 [S, max_blocks] CPU tensor, context_lens int32 [S] CPU tensor)."""
+        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
+        S = ids.numel()
+        if tables is None:
+            tables = torch.empty((S, max_blocks_per_seq), dtype=torch.int32)
+        if lens is None:
+            lens = torch.empty((S,), dtype=torch.int32)
+        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+        _check(self._lib.pa_build_block_tables(self._h, i32(ids), S, i32(tables), max_blocks_per_seq, i32(lens)))
+        return tables, lens

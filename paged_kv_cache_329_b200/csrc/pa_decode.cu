@@ -1,0 +1,976 @@
+// Paged decode attention for sm_100a.
+//
+// What is computed ("PagedAttention原理", "为什么会有 KV cache", eq. o_t = softmax(q_t K^T/sqrt(d)) V,
+// and "实现一个虚拟内存", eqs. K_j, V_j, A_ij, o_i): for each sequence and query head, the scores of
+// the query against the c cached keys, their softmax, and the softmax-weighted sum of the cached
+// values, where token t lives in physical block block_tables[s][t / B] at offset t % B.  The
+// denominator of A_ij is a sum over blocks, so it is accumulated block by block with a running
+// maximum (online softmax) and, across partitions of the context, merged by log-sum-exp.
+//
+// Design (one B200, HBM-bound: each cached token of each kv head is read once per step):
+//   * Work unit = (sequence, kv head, partition of P tokens).  A plan kernel lists the units
+//     (whole partitions first, then the tails); a persistent grid pulls them from an atomic
+//     counter, so long and short sequences balance across the 148 SMs.
+//   * Per CTA one producer warp streams 64-token tiles of K and V into shared memory with 2-D TMA
+//     loads (one box per physical block and 128-byte column panel, 128-byte swizzle), into a ring
+//     of stages guarded by full/empty mbarriers.  The q rows of the unit's head group come in with
+//     the first tile by a 1-D bulk copy.  Each block is located through the block table, so the
+//     kernel never touches a slot past the sequence's length.
+//   * Four consumer warps share every loaded tile across the g = H/Hk query heads of the group.
+//     q.k: each group of L lanes covers one token row (one 16-byte chunk per lane, q for that
+//     chunk held in registers), partial dot products are reduce-scattered across the L lanes so
+//     each lane ends with whole scores.  Online softmax in fp32 (log2 domain), then p.V: the same
+//     lanes own the same chunks of V and accumulate g output rows.
+//   * At the end of a unit the four warps merge their (max, sum, accumulator) states in shared
+//     memory in a fixed order, then write the final row (single-partition sequences) or the
+//     partial state for the combine kernel.  All summation orders depend only on logical token
+//     positions, so outputs do not change when blocks move to other physical ids.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace {
+
+using pa::ChunkTraits;
+
+constexpr int kTileTokens = 64;     // tokens per pipeline stage
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kPlanThreads = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Workspace header words.
+constexpr int kHdrCounter = 0;
+constexpr int kHdrNumItems = 1;
+constexpr int kHdrError = 2;
+constexpr size_t kHdrBytes = 256;
+
+enum : int { kFirst = 1, kLast = 2, kDone = 4, kSingle = 8 };
+
+struct __align__(16) StageMeta {
+  int s, kh, part, ntok, flags, pad0, pad1, pad2;
+};
+
+struct DecodeArgs {
+  const void* q;
+  void* out;
+  int out_dtype;
+  const int32_t* bt;
+  const int32_t* lens;
+  int S, H, Hk, max_blocks, n_blocks, B, P;
+  int max_c;         // context lengths are clamped to this (max_context_len)
+  float scale_log2;  // scale * log2(e)
+  const int2* items;
+  int* hdr;
+  float* part_o;
+  float* part_m;
+  float* part_l;
+  int max_parts;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- workspace layout ---------------------------------------------------------------------------
+
+struct WsLayout {
+  size_t items, part_m, part_l, part_o, total;
+};
+
+WsLayout ws_layout(int S, int H, int Hk, int d, int max_parts) {
+  WsLayout w;
+  size_t off = kHdrBytes;
+  w.items = off;
+  off = align_up(off + sizeof(int2) * static_cast<size_t>(S) * Hk * max_parts, 256);
+  w.part_m = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(S) * H * max_parts, 256);
+  w.part_l = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(S) * H * max_parts, 256);
+  w.part_o = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(S) * H * max_parts * d, 256);
+  w.total = off;
+  return w;
+}
+
+// ---- plan: list the work units -----------------------------------------------------------------
+// Unit order: every whole partition (parts 0 .. n_parts-2 of each sequence), ordered by
+// (sequence, part, kv head), then every sequence's last partition, ordered by (sequence, kv head).
+// n_parts(s) = max(1, ceil(c / P)); c = 0 still gets one unit, which writes zeros.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ lens, int S, int Hk, int P,
+                                                            int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
+  __shared__ int warp_tot[kPlanThreads / 32];
+  __shared__ int chunk_total;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  int base = 0;  // whole partitions listed so far (in units of (s, part), before the Hk factor)
+  for (int s0 = 0; s0 < S; s0 += kPlanThreads) {
+    const int s = s0 + tid;
+    int f = 0;
+    if (s < S) {
+      const int c = min(max(lens[s], 0), max_c);
+      f = max(1, (c + P - 1) / P) - 1;
+    }
+    int incl = f;  // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      int t = lane < kPlanThreads / 32 ? warp_tot[lane] : 0;
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) ti += v;
+      }
+      if (lane < kPlanThreads / 32) warp_tot[lane] = ti - t;  // exclusive prefix of warp totals
+      if (lane == 31) chunk_total = ti;
+    }
+    __syncthreads();
+    const int excl = base + warp_tot[wid] + incl - f;
+    for (int part = 0; part < f; ++part)
+      for (int kh = 0; kh < Hk; ++kh)
+        items[static_cast<size_t>(excl + part) * Hk + kh] = make_int2(s, (kh << 16) | part);
+    base += chunk_total;
+    __syncthreads();
+  }
+  const size_t n_full = static_cast<size_t>(base) * Hk;
+  bool clamped = false;
+  for (int s = tid; s < S; s += kPlanThreads) {
+    clamped |= lens[s] > max_c;
+    const int c = min(max(lens[s], 0), max_c);
+    const int last = max(1, (c + P - 1) / P) - 1;
+    for (int kh = 0; kh < Hk; ++kh) items[n_full + static_cast<size_t>(s) * Hk + kh] = make_int2(s, (kh << 16) | last);
+  }
+  const int any_clamped = __syncthreads_or(clamped);
+  if (tid == 0) {
+    hdr[kHdrCounter] = 0;
+    hdr[kHdrNumItems] = static_cast<int>(n_full) + S * Hk;
+    hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
+  }
+}
+
+// ---- the decode kernel --------------------------------------------------------------------------
+
+template <class T, int D, int G>
+struct Cfg {
+  static constexpr int kES = sizeof(T);
+  static constexpr int kE = ChunkTraits<T>::kElems;          // elements per 16-byte chunk
+  static constexpr int kCH = D / kE;                          // chunks per row
+  static constexpr int kPanelElems = 128 / kES;               // elements per 128-byte panel row
+  static constexpr int kNPanel = D / kPanelElems;             // panels per row
+  static constexpr int kPanelBytes = kTileTokens * 128;       // one panel of one tile
+  static constexpr int kKVBytes = kNPanel * kPanelBytes;      // K (or V) tile
+  static constexpr int kStageBytes = 2 * kKVBytes;
+  static constexpr int kStages = kNPanel == 1 ? 6 : 3;
+  static constexpr int kQBytes = G * D * kES;
+  static constexpr int kQSlot = (kQBytes + 127) / 128 * 128;
+  static constexpr int kL = kCH < 16 ? kCH : 16;              // lanes per token row
+  static constexpr int kCPL = kCH / kL;                       // chunks per lane
+  static constexpr int kNG = 32 / kL;                         // token groups per warp
+  static constexpr int kR = (G >= 8 || kL < 16) ? 4 : 8;      // tokens per group per pass
+  static constexpr int kTPW = kNG * kR;                       // tokens per warp per pass
+  static constexpr int kPasses = kTileTokens / (kConsumerWarps * kTPW);
+  static constexpr int kAcc = kCPL * kE;                      // accumulator floats per head per lane
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int kOffQ = kStages * kStageBytes;
+  static constexpr int kOffMeta = kOffQ + kStages * kQSlot;
+  static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(StageMeta));
+  static constexpr int kOffML = (kOffBar + (2 * kStages + 1) * 8 + 127) / 128 * 128;
+  static constexpr int kOffMerge = (kOffML + kConsumerWarps * G * 2 * 4 + 127) / 128 * 128;
+  static constexpr int kSmemBytes = kOffMerge + 2 * G * D * 4 + 1024;  // + alignment slack
+  static_assert(kPasses >= 1 && kTileTokens % (kConsumerWarps * kTPW) == 0, "tile/mapping mismatch");
+  static_assert(kCH % kL == 0, "chunks must split evenly over lanes");
+  static_assert(kQBytes % 16 == 0, "q rows must be whole 16-byte chunks");
+};
+
+// Reduce-scatter of partial dot products over the L lanes of a token group: at each level with
+// N > 1 tokens, a lane keeps half of them and adds its partner's partials for that half; once a
+// lane holds one token, the remaining levels add the partner's partial for the same token.
+template <int G, int R, int MSK, int N>
+__device__ __forceinline__ void reduce_scatter(float (&part)[G][R], int l) {
+  if constexpr (MSK >= 1) {
+    if constexpr (N > 1) {
+      constexpr int HALF = N / 2;
+      const bool up = (l & MSK) != 0;
+#pragma unroll
+      for (int j = 0; j < HALF; ++j)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float send = up ? part[h][j] : part[h][j + HALF];
+          const float keep = up ? part[h][j + HALF] : part[h][j];
+          part[h][j] = keep + __shfl_xor_sync(0xffffffffu, send, MSK);
+        }
+      reduce_scatter<G, R, MSK / 2, HALF>(part, l);
+    } else {
+#pragma unroll
+      for (int h = 0; h < G; ++h) part[h][0] += __shfl_xor_sync(0xffffffffu, part[h][0], MSK);
+      reduce_scatter<G, R, MSK / 2, 1>(part, l);
+    }
+  }
+}
+
+// Token (0..R-1) whose score lane l of a group holds after reduce_scatter, and the inverse.
+template <int L, int R>
+__device__ __forceinline__ int token_of_lane(int l) {
+  int t = 0, n = R;
+#pragma unroll
+  for (int msk = L / 2; msk >= 1; msk >>= 1)
+    if (n > 1) {
+      n >>= 1;
+      if (l & msk) t += n;
+    }
+  return t;
+}
+
+template <int L, int R>
+__device__ __forceinline__ int lane_of_token(int t) {
+  int l = 0, n = R;
+#pragma unroll
+  for (int msk = L / 2; msk >= 1; msk >>= 1)
+    if (n > 1) {
+      n >>= 1;
+      if (t & n) l |= msk;
+    }
+  return l;
+}
+
+// Lanes that hold a duplicate score (set bits at the all-reduce levels) do not add to the sum.
+template <int L, int R>
+__device__ __forceinline__ bool primary_lane(int l) {
+  int n = R, dup = 0;
+#pragma unroll
+  for (int msk = L / 2; msk >= 1; msk >>= 1) {
+    if (n > 1) n >>= 1;
+    else dup |= msk;
+  }
+  return (l & dup) == 0;
+}
+
+template <class OutT, int D, int G, int AC, int L, int CPL, int E>
+__device__ __forceinline__ void write_rows(OutT* base, const float (&acc)[G][AC], const float* mul, int l) {
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      float v[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = acc[h][k * E + e] * mul[h];
+      pa::store_floats<OutT, E>(base + static_cast<size_t>(h) * D + (k * L + l) * E, v);
+    }
+}
+
+template <class T, int D, int G>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                          const __grid_constant__ CUtensorMap tmV,
+                                                          const DecodeArgs a) {
+  using C = Cfg<T, D, G>;
+  constexpr int E = C::kE, L = C::kL, CPL = C::kCPL, NG = C::kNG, R = C::kR, AC = C::kAcc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* qslots = smem + C::kOffQ;
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + C::kOffMeta);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* epi = empty + C::kStages;  // consumer-only barrier for the end-of-unit merge
+  float* ml = reinterpret_cast<float*>(smem + C::kOffML);        // [warp][G][2] (max, sum)
+  float* merge = reinterpret_cast<float*>(smem + C::kOffMerge);  // [2][G][D]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      pa::mbar_init(&full[i], 1);
+      pa::mbar_init(&empty[i], kConsumerWarps);
+    }
+    pa::mbar_init(epi, kConsumerWarps * 32);
+    pa::fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ================================ producer warp ==========================================
+    if (lane == 0) {
+      pa::prefetch_tmap(&tmK);
+      pa::prefetch_tmap(&tmV);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;  // stages filled so far (for draining after a timeout)
+    const int n_items = a.hdr[kHdrNumItems];
+    bool ok = true;
+    while (ok) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(a.hdr + kHdrCounter, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      if (k >= n_items) {
+        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        if (lane == 0) {
+          meta[stage].flags = kDone;
+          pa::mbar_arrive(&full[stage]);
+        }
+        break;
+      }
+      const int2 it = a.items[k];
+      const int s = it.x, kh = it.y >> 16, part = it.y & 0xffff;
+      const int c = min(max(a.lens[s], 0), a.max_c);
+      const int n_parts = max(1, (c + a.P - 1) / a.P);
+      const int t0 = part * a.P;
+      const int t1 = min(t0 + a.P, c);
+      const int ntok_item = max(t1 - t0, 0);
+      const int ntiles = max(1, (ntok_item + kTileTokens - 1) / kTileTokens);
+      const int32_t* bt_row = a.bt + static_cast<size_t>(s) * a.max_blocks;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        const int tok0 = t0 + tile * kTileTokens;
+        const int ntok = max(0, min(kTileTokens, t1 - tok0));
+        const int nblk = (ntok + a.B - 1) / a.B;
+        const int j0 = tok0 / a.B;
+        int phys = -1;
+        if (lane < nblk) {
+          phys = __ldg(bt_row + j0 + lane);
+          if (phys < 0 || phys >= a.n_blocks) {
+            atomicOr(a.hdr + kHdrError, pa::kErrBadBlock);
+            phys = -1;  // a fully out-of-range box: the TMA unit fills it with zeros
+          }
+        }
+        const uint32_t bytes = static_cast<uint32_t>(nblk) * a.B * D * C::kES * 2u + (tile == 0 ? C::kQBytes : 0u);
+        if (lane == 0) {
+          StageMeta m;
+          m.s = s;
+          m.kh = kh;
+          m.part = part;
+          m.ntok = ntok;
+          m.flags = (tile == 0 ? kFirst : 0) | (tile == ntiles - 1 ? kLast : 0) | (n_parts == 1 ? kSingle : 0);
+          meta[stage] = m;
+          pa::mbar_arrive_expect_tx(&full[stage], bytes);
+        }
+        __syncwarp();
+        uint8_t* kdst = stages + stage * C::kStageBytes;
+        uint8_t* vdst = kdst + C::kKVBytes;
+        if (lane < nblk) {
+          const int y = (phys * a.Hk + kh) * a.B;
+#pragma unroll
+          for (int p = 0; p < C::kNPanel; ++p) {
+            pa::tma_load_2d(kdst + p * C::kPanelBytes + lane * a.B * 128, &tmK, p * C::kPanelElems, y, &full[stage]);
+            pa::tma_load_2d(vdst + p * C::kPanelBytes + lane * a.B * 128, &tmV, p * C::kPanelElems, y, &full[stage]);
+          }
+        }
+        if (tile == 0 && lane == 0) {
+          const uint8_t* qsrc = static_cast<const uint8_t*>(a.q) +
+                                (static_cast<size_t>(s) * a.H + static_cast<size_t>(kh) * G) * D * C::kES;
+          pa::bulk_load(qslots + stage * C::kQSlot, qsrc, C::kQBytes, &full[stage]);
+        }
+        ++issued;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      // Let every copy this warp started land before the CTA can exit.
+      int st = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < C::kStages && i < issued; ++i) {
+        if (--st < 0) {
+          st = C::kStages - 1;
+          ph ^= 1;
+        }
+        pa::mbar_wait(&full[st], ph);
+      }
+    }
+    return;
+  }
+
+  // ================================== consumer warps ============================================
+  const int grp = lane / L, l = lane % L;
+  const int my_tok = token_of_lane<L, R>(l);
+  const bool primary = primary_lane<L, R>(l);
+  float qf[G][AC];
+  float acc[G][AC];
+  float m_run[G], l_lane[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_run[h] = -INFINITY;
+    l_lane[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < AC; ++e) acc[h][e] = 0.f, qf[h][e] = 0.f;
+  }
+
+  int stage = 0;
+  uint32_t phase = 0, epi_phase = 0;
+  // All 128 consumer threads arrive; a wait that runs out of time abandons the kernel.
+  auto epi_sync = [&]() -> bool {
+    pa::mbar_arrive(epi);
+    const bool done = pa::mbar_wait(epi, epi_phase);
+    epi_phase ^= 1;
+    if (!done && lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    return done;
+  };
+  while (true) {
+    if (!pa::mbar_wait(&full[stage], phase)) {
+      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      return;
+    }
+    const StageMeta mt = meta[stage];
+    if (mt.flags & kDone) break;
+    const uint8_t* ks = stages + stage * C::kStageBytes;
+    const uint8_t* vs = ks + C::kKVBytes;
+    const int ntok = mt.ntok;
+
+    if (mt.flags & kFirst) {
+      const T* qsm = reinterpret_cast<const T*>(qslots + stage * C::kQSlot);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(qsm + h * D + (k * L + l) * E);
+          ChunkTraits<T>::to_float(raw, &qf[h][k * E]);
+        }
+#pragma unroll
+        for (int e = 0; e < AC; ++e) qf[h][e] *= a.scale_log2;
+        m_run[h] = -INFINITY;
+        l_lane[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < AC; ++e) acc[h][e] = 0.f;
+      }
+    }
+
+#pragma unroll
+    for (int pass = 0; pass < C::kPasses; ++pass) {
+      const int row0 = pass * (kConsumerWarps * C::kTPW) + warp * C::kTPW + grp * R;
+      // ---- scores: partial dot products over this lane's chunks, then reduce-scatter ----
+      float part[G][R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) part[h][i] = 0.f;
+        const int row = row0 + i;
+        if (row < ntok) {
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const int c = k * L + l;
+            const uint4 raw =
+                pa::lds128(ks + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+            float kv[E];
+            ChunkTraits<T>::to_float(raw, kv);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int e = 0; e < E; ++e) part[h][i] = fmaf(qf[h][k * E + e], kv[e], part[h][i]);
+          }
+        }
+      }
+      reduce_scatter<G, R, L / 2, R>(part, l);
+
+      // ---- online softmax (scores are in log2 units) ----
+      const bool valid = row0 + my_tok < ntok;
+      float sc[G], mt_[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        sc[h] = valid ? part[h][0] : -INFINITY;
+        mt_[h] = sc[h];
+      }
+#pragma unroll
+      for (int msk = 16; msk >= 1; msk >>= 1) {
+        // lanes that differ only in all-reduce bits hold the same score; skip those levels
+        const bool dup_level = (msk < L) && (msk < L / R);
+        if (!dup_level) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) mt_[h] = fmaxf(mt_[h], __shfl_xor_sync(0xffffffffu, mt_[h], msk));
+        }
+      }
+      float p[G];
+      bool rescale = false;
+      float alpha[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mn = fmaxf(m_run[h], mt_[h]);
+        alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[h] - mn);
+        p[h] = (mn == -INFINITY) ? 0.f : exp2f(sc[h] - mn);
+        rescale |= (mn != m_run[h]);
+        m_run[h] = mn;
+        l_lane[h] = l_lane[h] * alpha[h] + (primary ? p[h] : 0.f);
+      }
+      if (rescale) {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < AC; ++e) acc[h][e] *= alpha[h];
+      }
+
+      // ---- p.V over the group's R tokens ----
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int src = grp * L + lane_of_token<L, R>(i);
+        float pi[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) pi[h] = __shfl_sync(0xffffffffu, p[h], src);
+        const int row = row0 + i;
+        if (row < ntok) {
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const int c = k * L + l;
+            const uint4 raw =
+                pa::lds128(vs + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+            float vv[E];
+            ChunkTraits<T>::to_float(raw, vv);
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int e = 0; e < E; ++e) acc[h][k * E + e] = fmaf(pi[h], vv[e], acc[h][k * E + e]);
+          }
+        }
+      }
+    }
+
+    __syncwarp();
+    if (lane == 0) pa::mbar_arrive(&empty[stage]);
+
+    if (mt.flags & kLast) {
+      // ---- merge the four warps' states in a fixed order and write the result ----
+      float lw[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = l_lane[h];
+#pragma unroll
+        for (int msk = 16; msk >= 1; msk >>= 1) v += __shfl_xor_sync(0xffffffffu, v, msk);
+        lw[h] = v;
+      }
+#pragma unroll
+      for (int msk = L; msk < 32; msk <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < AC; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], msk);
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          ml[(warp * G + h) * 2] = m_run[h];
+          ml[(warp * G + h) * 2 + 1] = lw[h];
+        }
+      }
+      if (!epi_sync()) return;
+      float M[G], den[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, ml[(w * G + h) * 2]);
+        float dsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = ml[(w * G + h) * 2];
+          if (mw != -INFINITY) dsum += exp2f(mw - mx) * ml[(w * G + h) * 2 + 1];
+        }
+        M[h] = mx;
+        den[h] = dsum;
+        const float mine = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mx);
+#pragma unroll
+        for (int e = 0; e < AC; ++e) acc[h][e] *= mine;
+      }
+      // tree sum: (w0 + w2) + (w1 + w3), then w0 + w1; lanes of group 0 hold the warp's sums
+      const bool writer = grp == 0;
+      constexpr unsigned kWriterMask = L == 32 ? 0xffffffffu : ((1u << L) - 1u);
+      if (warp >= 2 && writer) {
+        float* buf = merge + (warp - 2) * G * D;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int e = 0; e < E; e += 4)
+              *reinterpret_cast<float4*>(buf + h * D + (k * L + l) * E + e) =
+                  make_float4(acc[h][k * E + e], acc[h][k * E + e + 1], acc[h][k * E + e + 2], acc[h][k * E + e + 3]);
+      }
+      if (!epi_sync()) return;
+      if (warp < 2 && writer) {
+        float* buf = merge + warp * G * D;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(buf + h * D + (k * L + l) * E + e);
+              acc[h][k * E + e] += v.x;
+              acc[h][k * E + e + 1] += v.y;
+              acc[h][k * E + e + 2] += v.z;
+              acc[h][k * E + e + 3] += v.w;
+            }
+        if (warp == 1) {
+          __syncwarp(kWriterMask);  // only the writer lanes are here
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int k = 0; k < CPL; ++k)
+#pragma unroll
+              for (int e = 0; e < E; e += 4)
+                *reinterpret_cast<float4*>(buf + h * D + (k * L + l) * E + e) = make_float4(
+                    acc[h][k * E + e], acc[h][k * E + e + 1], acc[h][k * E + e + 2], acc[h][k * E + e + 3]);
+        }
+      }
+      if (!epi_sync()) return;
+      if (warp == 0 && writer) {
+        const float* buf = merge + G * D;
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int k = 0; k < CPL; ++k)
+#pragma unroll
+            for (int e = 0; e < E; e += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(buf + h * D + (k * L + l) * E + e);
+              acc[h][k * E + e] += v.x;
+              acc[h][k * E + e + 1] += v.y;
+              acc[h][k * E + e + 2] += v.z;
+              acc[h][k * E + e + 3] += v.w;
+            }
+        const size_t row = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;
+        if (mt.flags & kSingle) {
+          float inv[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) inv[h] = den[h] > 0.f ? 1.f / den[h] : 0.f;
+          if (a.out_dtype == PA_F32)
+            write_rows<float, D, G, AC, L, CPL, E>(static_cast<float*>(a.out) + row * D, acc, inv, l);
+          else if (a.out_dtype == PA_F16)
+            write_rows<__half, D, G, AC, L, CPL, E>(static_cast<__half*>(a.out) + row * D, acc, inv, l);
+          else
+            write_rows<__nv_bfloat16, D, G, AC, L, CPL, E>(static_cast<__nv_bfloat16*>(a.out) + row * D, acc, inv,
+                                                           l);
+        } else {
+          float one[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h) one[h] = 1.f;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const size_t pidx = (row + h) * a.max_parts + mt.part;
+            float acc_h[1][AC];
+#pragma unroll
+            for (int e = 0; e < AC; ++e) acc_h[0][e] = acc[h][e];
+            write_rows<float, D, 1, AC, L, CPL, E>(a.part_o + pidx * D, acc_h, one, l);
+            if (l == 0) {
+              a.part_m[pidx] = M[h] == -INFINITY ? -INFINITY : M[h] * kLn2;
+              a.part_l[pidx] = den[h];
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m_run[h] = -INFINITY;
+        l_lane[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < AC; ++e) acc[h][e] = 0.f;
+      }
+    }
+
+    if (++stage == C::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+}
+
+// ---- log-sum-exp combine -----------------------------------------------------------------------
+// One warp per (sequence, query head); lane owns D/32 consecutive dims.  Sequences with fewer
+// than min_parts partitions are skipped (the decode kernel already wrote them).
+template <class OutT, int D>
+__global__ void __launch_bounds__(256) combine_kernel(OutT* __restrict__ out, const float* __restrict__ part_o,
+                                                      const float* __restrict__ part_m,
+                                                      const float* __restrict__ part_l,
+                                                      const int32_t* __restrict__ lens, int S, int H,
+                                                      int max_parts, int P, int min_parts) {
+  // Partitions past max_parts are never read: a length that needs more is cut to max_parts * P.
+  constexpr int PER = D / 32;
+  const long long gw = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(S) * H) return;
+  const int s = static_cast<int>(gw / H);
+  const int c = max(lens[s], 0);
+  const int np = min((c + P - 1) / P, max_parts);
+  OutT* o = out + gw * D + lane * PER;
+  float res[PER];
+  if (np == 0) {  // empty context: zeros (the decode kernel already wrote them when min_parts > 1)
+    if (min_parts <= 1) {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) res[e] = 0.f;
+      pa::store_pairs<OutT, PER>(o, res);
+    }
+    return;
+  }
+  if (np < min_parts) return;
+  const float* pm = part_m + gw * max_parts;
+  const float* pl = part_l + gw * max_parts;
+  float mx = -INFINITY;
+  for (int p = lane; p < np; p += 32) mx = fmaxf(mx, pm[p]);
+#pragma unroll
+  for (int msk = 16; msk >= 1; msk >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float den = 0.f;
+  if (mx != -INFINITY) {
+    for (int p = 0; p < np; ++p) {
+      const float mp = pm[p];
+      if (mp == -INFINITY) continue;
+      const float w = expf(mp - mx);
+      den = fmaf(w, pl[p], den);
+      const float* src = part_o + (gw * max_parts + p) * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; e += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(src + e);
+        acc[e] = fmaf(w, v.x, acc[e]);
+        acc[e + 1] = fmaf(w, v.y, acc[e + 1]);
+      }
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) res[e] = acc[e] * inv;
+  pa::store_pairs<OutT, PER>(o, res);
+}
+
+template <int D>
+cudaError_t launch_combine(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
+                           const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
+                           cudaStream_t st) {
+  const long long threads = static_cast<long long>(S) * H * 32;
+  const int grid = static_cast<int>((threads + 255) / 256);
+  if (grid == 0) return cudaSuccess;
+  if (out_dtype == PA_F32)
+    combine_kernel<float, D><<<grid, 256, 0, st>>>(static_cast<float*>(out), po, pm, pl, lens, S, H, max_parts, P, min_parts);
+  else if (out_dtype == PA_F16)
+    combine_kernel<__half, D><<<grid, 256, 0, st>>>(static_cast<__half*>(out), po, pm, pl, lens, S, H, max_parts, P, min_parts);
+  else
+    combine_kernel<__nv_bfloat16, D><<<grid, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), po, pm, pl, lens, S, H, max_parts, P,
+                                                           min_parts);
+  return cudaGetLastError();
+}
+
+// ---- host side ----------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a cache viewed as [n_blocks*Hk*B rows][d]; box = B rows x 128 bytes.
+bool make_cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long long rows, int B) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  const CUtensorMapDataType t = dt == PA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int es = static_cast<int>(pa::elem_size(dt));
+  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * es};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(B)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, t, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+DeviceInfo device_info() {
+  DeviceInfo di;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (di.sms <= 0) di.sms = 148;
+  return di;
+}
+
+template <class T, int D, int G>
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int max_units,
+                          cudaStream_t st) {
+  using C = Cfg<T, D, G>;
+  static int occupancy = -1;  // per instantiation; device properties are uniform on a B200 node
+  cudaError_t e = cudaSuccess;
+  if (occupancy < 0) {
+    e = cudaFuncSetAttribute(decode_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<T, D, G>, kThreads, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    occupancy = occ < 1 ? 1 : occ;
+  }
+  const DeviceInfo di = device_info();
+  long long grid = static_cast<long long>(di.sms) * occupancy;
+  if (grid > max_units) grid = max_units;
+  if (grid < 1) grid = 1;
+  decode_kernel<T, D, G><<<static_cast<int>(grid), kThreads, C::kSmemBytes, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+template <class T, int D>
+cudaError_t dispatch_g(int g, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int max_units,
+                       cudaStream_t st) {
+  switch (g) {
+    case 1: return launch_decode<T, D, 1>(tk, tv, a, max_units, st);
+    case 2: return launch_decode<T, D, 2>(tk, tv, a, max_units, st);
+    case 4: return launch_decode<T, D, 4>(tk, tv, a, max_units, st);
+    default: return launch_decode<T, D, 8>(tk, tv, a, max_units, st);
+  }
+}
+
+template <class T>
+cudaError_t dispatch_d(int d, int g, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                       int max_units, cudaStream_t st) {
+  return d == 64 ? dispatch_g<T, 64>(g, tk, tv, a, max_units, st) : dispatch_g<T, 128>(g, tk, tv, a, max_units, st);
+}
+
+int default_partition(int S, int Hk, int max_context_len) {
+  // Whole 512-token partitions keep the partial-state traffic small (under 2% of the KV bytes
+  // at d = 128); with few (sequence, kv head) pairs, shorter partitions give every SM work.
+  const long long units512 = static_cast<long long>(S) * Hk * ((max_context_len + 511) / 512);
+  if (units512 >= 4 * 148) return 512;
+  return 256;
+}
+
+int max_parts_for(int max_context_len, int P) {
+  const int n = (max_context_len + P - 1) / P;
+  return n < 1 ? 1 : n;
+}
+
+}  // namespace
+
+extern "C" int pa_decode_default_partition(int S, int Hk, int max_context_len) {
+  return default_partition(S, Hk, max_context_len);
+}
+
+extern "C" size_t pa_decode_workspace_size(int S, int H, int Hk, int d, int max_context_len, int partition_size) {
+  if (S < 0 || H <= 0 || Hk <= 0 || d <= 0 || max_context_len < 0) return 0;
+  const int P = partition_size > 0 ? partition_size : default_partition(S, Hk, max_context_len);
+  return ws_layout(S, H, Hk, d, max_parts_for(max_context_len, P)).total;
+}
+
+extern "C" pa_status pa_workspace_error(const void* workspace, int* flags, void* stream) {
+  if (!workspace || !flags) return pa::fail(PA_ERR_INVALID_ARG, "pa_workspace_error: null argument");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(flags, static_cast<const int*>(workspace) + kHdrError, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_workspace_error: %s", cudaGetErrorString(e));
+  return pa::ok();
+}
+
+extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                               int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq,
+                               int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (S < 0 || H <= 0 || Hk <= 0 || n_blocks <= 0 || max_blocks_per_seq < 0 || max_context_len < 0)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: bad sizes (S=%d H=%d Hk=%d n_blocks=%d)", S, H, Hk, n_blocks);
+  if (H % Hk != 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: H (%d) must be a multiple of Hk (%d)", H, Hk);
+  const int g = H / Hk;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: H/Hk = %d not in {1,2,4,8}", g);
+  if (d != 64 && d != 128) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: d = %d not in {64,128}", d);
+  if (B != 8 && B != 16 && B != 32) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: B = %d not in {8,16,32}", B);
+  if (!pa::valid_dtype(kv_dtype) || !pa::valid_dtype(out_dtype)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: unknown dtype");
+  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: scale must be finite");
+  const int P = partition_size > 0 ? partition_size : default_partition(S, Hk, max_context_len);
+  if (P % kTileTokens != 0 || P > (1 << 24)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: partition_size %d must be a positive multiple of 64", P);
+  const int max_parts = max_parts_for(max_context_len, P);
+  if (max_parts > 0xffff) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: more than 65535 partitions per sequence");
+  if (static_cast<long long>(max_blocks_per_seq) * B < max_context_len)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: max_blocks_per_seq * B < max_context_len");
+  const long long rows = static_cast<long long>(n_blocks) * Hk * B;
+  if (rows >= (1ll << 31) || static_cast<long long>(S) * Hk * max_parts > (1ll << 31))
+    return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: problem too large for 32-bit indices");
+  if (S == 0) return pa::ok();
+  if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: null pointer");
+  if (!pa::aligned16(out) || !pa::aligned16(query) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: workspace must be 256-byte aligned");
+  const WsLayout wl = ws_layout(S, H, Hk, d, max_parts);
+  if (workspace_bytes < wl.total)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: workspace of %zu bytes < %zu needed", workspace_bytes, wl.total);
+
+  CUtensorMap tk, tv;
+  if (!make_cache_map(&tk, k_cache, kv_dtype, d, rows, B) || !make_cache_map(&tv, v_cache, kv_dtype, d, rows, B))
+    return pa::fail(PA_ERR_CUDA, "pa_decode: could not encode the cache tensor maps");
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeArgs a;
+  a.q = query;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.bt = block_tables;
+  a.lens = context_lens;
+  a.S = S;
+  a.H = H;
+  a.Hk = Hk;
+  a.max_blocks = max_blocks_per_seq;
+  a.n_blocks = n_blocks;
+  a.B = B;
+  a.P = P;
+  a.max_c = max_context_len;
+  a.scale_log2 = scale * kLog2e;
+  a.items = reinterpret_cast<const int2*>(ws + wl.items);
+  a.hdr = reinterpret_cast<int*>(ws);
+  a.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+  a.part_m = reinterpret_cast<float*>(ws + wl.part_m);
+  a.part_l = reinterpret_cast<float*>(ws + wl.part_l);
+  a.max_parts = max_parts;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  plan_kernel<<<1, kPlanThreads, 0, st>>>(context_lens, S, Hk, P, max_context_len, reinterpret_cast<int2*>(ws + wl.items), a.hdr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: plan launch failed: %s", cudaGetErrorString(e));
+
+  const long long units = static_cast<long long>(S) * Hk * max_parts;
+  const int max_units = static_cast<int>(units < (1ll << 30) ? units : (1ll << 30));
+  if (kv_dtype == PA_F32) e = dispatch_d<float>(d, g, tk, tv, a, max_units, st);
+  else if (kv_dtype == PA_F16) e = dispatch_d<__half>(d, g, tk, tv, a, max_units, st);
+  else e = dispatch_d<__nv_bfloat16>(d, g, tk, tv, a, max_units, st);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s", cudaGetErrorString(e));
+
+  if (max_parts > 1) {
+    e = d == 64 ? launch_combine<64>(out, out_dtype, a.part_o, a.part_m, a.part_l, context_lens, S, H, max_parts, P, 2, st)
+                : launch_combine<128>(out, out_dtype, a.part_o, a.part_m, a.part_l, context_lens, S, H, max_parts, P, 2, st);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: combine launch failed: %s", cudaGetErrorString(e));
+  }
+  return pa::ok();
+}
+
+extern "C" pa_status pa_combine(void* out, pa_dtype out_dtype, const float* part_o, const float* part_m,
+                                const float* part_l, const int32_t* context_lens, int S, int H, int d, int max_parts,
+                                int partition_size, void* stream) {
+  if (S < 0 || H <= 0 || max_parts <= 0 || partition_size <= 0)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_combine: bad sizes");
+  if (d != 64 && d != 128) return pa::fail(PA_ERR_UNSUPPORTED, "pa_combine: d = %d not in {64,128}", d);
+  if (!pa::valid_dtype(out_dtype)) return pa::fail(PA_ERR_INVALID_ARG, "pa_combine: unknown dtype");
+  if (S == 0) return pa::ok();
+  if (!out || !part_o || !part_m || !part_l || !context_lens) return pa::fail(PA_ERR_INVALID_ARG, "pa_combine: null pointer");
+  if (!pa::aligned16(out) || !pa::aligned16(part_o)) return pa::fail(PA_ERR_INVALID_ARG, "pa_combine: out/part_o must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e =
+      d == 64 ? launch_combine<64>(out, out_dtype, part_o, part_m, part_l, context_lens, S, H, max_parts, partition_size, 1, st)
+              : launch_combine<128>(out, out_dtype, part_o, part_m, part_l, context_lens, S, H, max_parts, partition_size, 1, st);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_combine: launch failed: %s", cudaGetErrorString(e));
+  return pa::ok();
+}

@@ -1,0 +1,195 @@
+// Device helpers for libpa's sm_100a kernels: shared-memory barriers, TMA copies, bounded waits
+// and element conversions.  Every wait on a barrier is bounded in time: a wait that gives up
+// returns false and the caller records an error and leaves the kernel instead of spinning.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace pa {
+
+// Error bits written to the decode workspace's error word.
+constexpr int kErrBadBlock = 1;    // block-table entry outside [0, n_blocks): read as zeros
+constexpr int kErrWaitTimeout = 2; // a pipeline wait ran out of time
+constexpr int kErrBadLength = 4;   // a context length above max_context_len: cut to it
+
+// A pipeline wait that has not completed after this long is abandoned.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Makes barrier initialisation visible to the async (TMA) proxy; follow with __syncthreads().
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Waits for the phase of `bar` with the given parity to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return false;
+}
+
+// 2-D tiled TMA load of one box into shared memory; completion is counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Contiguous bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_addr(p)));
+  return v;
+}
+
+// ---- 16-byte chunk -> floats -------------------------------------------------------------------
+
+template <class T>
+struct ChunkTraits;
+
+template <>
+struct ChunkTraits<float> {
+  static constexpr int kElems = 4;
+  __device__ __forceinline__ static void to_float(const uint4& r, float* f) {
+    f[0] = __uint_as_float(r.x);
+    f[1] = __uint_as_float(r.y);
+    f[2] = __uint_as_float(r.z);
+    f[3] = __uint_as_float(r.w);
+  }
+};
+
+template <>
+struct ChunkTraits<__half> {
+  static constexpr int kElems = 8;
+  __device__ __forceinline__ static void to_float(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h2 = *reinterpret_cast<const __half2*>(&w[i]);
+      float2 v = __half22float2(h2);
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+  }
+};
+
+template <>
+struct ChunkTraits<__nv_bfloat16> {
+  static constexpr int kElems = 8;
+  // bfloat16 is the upper half of a binary32: widening is a shift or a mask.
+  __device__ __forceinline__ static void to_float(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+// ---- float -> output element --------------------------------------------------------------------
+
+template <class T>
+__device__ __forceinline__ T from_float(float x);
+template <>
+__device__ __forceinline__ float from_float<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __half from_float<__half>(float x) { return __float2half_rn(x); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Stores n (a multiple of 4) floats converted to T at p (16-byte aligned when n*sizeof(T) >= 16).
+template <class T, int N>
+__device__ __forceinline__ void store_floats(T* p, const float* v) {
+  static_assert(N % 4 == 0, "store_floats: N must be a multiple of 4");
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4)
+      *reinterpret_cast<float4*>(p + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      T t[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) t[j] = from_float<T>(v[i + j]);
+      *reinterpret_cast<uint2*>(p + i) = *reinterpret_cast<const uint2*>(t);
+    }
+  }
+}
+
+// Stores n (even) floats converted to T at p, two at a time (p aligned to 2 * sizeof(T)).
+template <class T, int N>
+__device__ __forceinline__ void store_pairs(T* p, const float* v) {
+  static_assert(N % 2 == 0, "store_pairs: N must be even");
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    if constexpr (sizeof(T) == 4) {
+      *reinterpret_cast<float2*>(p + i) = make_float2(v[i], v[i + 1]);
+    } else {
+      T t[2] = {from_float<T>(v[i]), from_float<T>(v[i + 1])};
+      *reinterpret_cast<uint32_t*>(p + i) = *reinterpret_cast<const uint32_t*>(t);
+    }
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,259 @@
+"""GPU parity of libpa's kernels against the fp64 oracle, through the C ABI.
+
+Tolerances (max-abs, on fp32 outputs of the same kernels): 1e-5 for fp32 inputs, 2e-3 for fp16 and
+bf16 inputs (fp32 accumulation).  Outputs in the input's 16-bit type are checked to within one
+unit in the last place of the oracle's value rounded to that type.  Cache writes, block copies and
+physical-permutation checks are bit-exact.
+"""
+import math
+
+import pytest
+import torch
+
+from paged_kv_cache_329_b200 import api
+from paged_kv_cache_329_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.float16: 2e-3, torch.bfloat16: 2e-3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from paged_kv_cache_329_b200 import build
+
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _run(case: W.DecodeCase, out_dtype=torch.float32, P=0, max_c=None):
+    dev = case.to("cuda") if not case.q.is_cuda else case
+    if max_c is None:
+        max_c = int(case.context_lens.max()) if case.S else 0
+    ws = api.alloc_workspace(case.S, case.H, case.Hk, case.d, max_c, P)
+    out = api.pa_decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                        max_context_len=max_c, scale=case.scale, out_dtype=out_dtype, partition_size=P,
+                        workspace=ws)
+    torch.cuda.synchronize()
+    assert api.workspace_error(ws) == 0
+    return out.cpu()
+
+
+def _oracle(oracle_mod, case, seqs=None):
+    """Oracle output for all sequences, or for a sample (gathering their blocks into a small pool)."""
+    q, bt, cl = case.q.cpu(), case.block_tables.cpu(), case.context_lens.cpu()
+    if seqs is None:
+        return oracle_mod.decode(q, case.k_cache.cpu(), case.v_cache.cpu(), bt, cl, case.scale, n_threads=0)
+    seqs = torch.as_tensor(seqs)
+    bt_s = bt[seqs]
+    used = torch.unique(bt_s[bt_s >= 0])
+    remap = torch.full((case.n_blocks,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(used.numel(), dtype=torch.int32)
+    bt_r = torch.where(bt_s >= 0, remap[bt_s.clamp(min=0).long()], bt_s)
+    kc = case.k_cache[used.to(case.k_cache.device)].cpu()
+    vc = case.v_cache[used.to(case.v_cache.device)].cpu()
+    return oracle_mod.decode(q[seqs], kc, vc, bt_r, cl[seqs], case.scale, n_threads=0)
+
+
+def _assert_close(got, ref, dtype, what=""):
+    assert torch.isfinite(got).all(), f"{what}: non-finite output"
+    err = (got.double() - ref).abs().max().item()
+    assert err <= TOL[dtype], f"{what}: max-abs error {err:.3g} > {TOL[dtype]}"
+    return err
+
+
+def _assert_ulp(got, ref, what=""):
+    """got: 16-bit output; ref: fp64 oracle.  |got - RNE(ref)| <= 1 ulp."""
+    want = ref.to(got.dtype)
+    gi = got.view(torch.int16).int()
+    wi = want.view(torch.int16).int()
+    ok = ((gi - wi).abs() <= 1) | ((got.double() - want.double()).abs() <= 1e-6)
+    assert ok.all(), f"{what}: {(~ok).sum().item()} elements differ by more than 1 ulp"
+
+
+# ---- the five serving scenarios ----------------------------------------------------------------
+
+def test_tiny_fp32(oracle_mod):
+    case = W.tiny_fp32()
+    ref = _oracle(oracle_mod, case)
+    _assert_close(_run(case), ref, torch.float32, "tiny_fp32")
+
+
+def test_mha13b_fp16_with_cache_write(oracle_mod):
+    case = W.mha13b_fp16()
+    tables, lens, slots = W.new_token_slots(case, W.generator(102))
+    g = W.generator(103)
+    key = W.randn(g, (case.S, case.Hk, case.d), torch.float16)
+    val = W.randn(g, (case.S, case.Hk, case.d), torch.float16)
+    k_ref, v_ref = oracle_mod.cache_write(case.k_cache, case.v_cache, key, val, slots)
+    dev = case.to("cuda")
+    api.pa_cache_write(dev.k_cache, dev.v_cache, key.cuda(), val.cuda(), slots.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(dev.k_cache.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(dev.v_cache.cpu().view(torch.int16), v_ref.view(torch.int16))
+    grown = W.DecodeCase(case.name, case.q, k_ref, v_ref, tables, lens, case.scale, case.H, case.Hk, case.d, case.B)
+    dev2 = W.DecodeCase(case.name, dev.q, dev.k_cache, dev.v_cache, tables.cuda(), lens.cuda(), case.scale,
+                        case.H, case.Hk, case.d, case.B)
+    ref = _oracle(oracle_mod, grown)
+    _assert_close(_run(dev2, max_c=int(lens.max())), ref, torch.float16, "mha13b_fp16")
+    _assert_ulp(_run(dev2, torch.float16, max_c=int(lens.max())), ref, "mha13b_fp16 fp16 out")
+
+
+def test_gqa8k_bf16_full_size_sampled(oracle_mod):
+    case = W.gqa8k_bf16(device="cuda")
+    lens = case.context_lens.cpu()
+    order = torch.argsort(lens)
+    sample = torch.unique(torch.cat([order[:6], order[-6:], torch.arange(0, case.S, 23)]))
+    ref = _oracle(oracle_mod, case, sample)
+    got = _run(case)
+    _assert_close(got[sample], ref, torch.bfloat16, "gqa8k_bf16")
+    got16 = _run(case, torch.bfloat16)
+    _assert_ulp(got16[sample], ref, "gqa8k_bf16 bf16 out")
+
+
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_long_context_full_size_sampled(oracle_mod, B):
+    case = W.long_bf16(B=B, device="cuda")
+    sample = [0, 7, int(torch.argmax(case.context_lens.cpu()))]
+    ref = _oracle(oracle_mod, case, sample)
+    for P in (256, 1024):
+        got = _run(case, P=P)
+        _assert_close(got[sample], ref, torch.bfloat16, f"long B={B} P={P}")
+
+
+# ---- edge cases ----------------------------------------------------------------------------------
+
+EDGE_LENS = [1, 7, 8, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 255, 256, 257, 511, 512, 513, 1100]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_edge_lengths(oracle_mod, dtype, g, d, B):
+    Hk = 2
+    case = W.paged_case("edge", EDGE_LENS, g * Hk, Hk, d, B, dtype, 1000 + g * 7 + d + B)
+    ref = _oracle(oracle_mod, case)
+    for P in (0, 64, 256):
+        _assert_close(_run(case, P=P), ref, dtype, f"{dtype} g={g} d={d} B={B} P={P}")
+
+
+def test_zero_length_sequences_give_zero(oracle_mod):
+    case = W.paged_case("zero", [0, 5, 0, 300, 0], 8, 2, 128, 16, torch.bfloat16, 77)
+    out = _run(case, P=64)
+    assert torch.count_nonzero(out[0]) == 0 and torch.count_nonzero(out[2]) == 0 and torch.count_nonzero(out[4]) == 0
+    _assert_close(out, _oracle(oracle_mod, case), torch.bfloat16, "zero lengths")
+
+
+def test_all_empty_batch():
+    case = W.paged_case("empty", [0, 0], 4, 4, 64, 16, torch.float16, 78)
+    assert torch.count_nonzero(_run(case)) == 0
+
+
+def test_output_types(oracle_mod):
+    case = W.paged_case("types", [3, 70, 600], 16, 4, 128, 16, torch.float16, 79)
+    ref = _oracle(oracle_mod, case)
+    _assert_close(_run(case, torch.float32), ref, torch.float16, "f32 out")
+    _assert_ulp(_run(case, torch.float16), ref, "f16 out")
+    _assert_ulp(_run(case, torch.bfloat16), ref, "bf16 out")
+
+
+# ---- determinism and placement -----------------------------------------------------------------
+
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_physical_permutation_is_bit_identical(B):
+    case = W.paged_case("perm", [1, B + 1, 200, 700, 1500], 32, 8, 128, B, torch.bfloat16, 80 + B, pool_factor=2.0)
+    o1 = _run(case, P=256)
+    n = case.n_blocks
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(B))
+    kc2 = torch.empty_like(case.k_cache)
+    vc2 = torch.empty_like(case.v_cache)
+    kc2[perm] = case.k_cache
+    vc2[perm] = case.v_cache
+    bt2 = case.block_tables.clone()
+    m = bt2 >= 0
+    bt2[m] = perm[bt2[m].long()].to(torch.int32)
+    case2 = W.DecodeCase("perm2", case.q, kc2, vc2, bt2, case.context_lens, case.scale, case.H, case.Hk, case.d, B)
+    o2 = _run(case2, P=256)
+    assert torch.equal(o1, o2)
+    assert torch.equal(o1, _run(case, P=256))  # and a repeat call
+
+
+def test_split_and_unsplit_agree(oracle_mod):
+    case = W.paged_case("split", [2000, 3000, 64, 4097], 32, 8, 128, 16, torch.bfloat16, 90)
+    ref = _oracle(oracle_mod, case)
+    outs = [_run(case, P=P) for P in (64, 512, 4160)]   # 4160 >= every length: no split at all
+    for o in outs:
+        _assert_close(o, ref, torch.bfloat16, "split")
+    assert (outs[0] - outs[2]).abs().max() < 1e-4
+
+
+def test_shared_prefix_reads_same_blocks(oracle_mod):
+    # Sequences whose tables share the prompt blocks and whose tails and queries match produce
+    # identical outputs.
+    case = W.paged_case("pref", [1030, 1030], 32, 8, 128, 16, torch.bfloat16, 91, sentinel="none", n_blocks=200)
+    bt = case.block_tables.clone()
+    bt[1, :64] = bt[0, :64]
+    kc, vc = case.k_cache.clone(), case.v_cache.clone()
+    kc[int(bt[1, 64])] = kc[int(bt[0, 64])]
+    vc[int(bt[1, 64])] = vc[int(bt[0, 64])]
+    q = case.q.clone()
+    q[1] = q[0]
+    c2 = W.DecodeCase("pref2", q, kc, vc, bt, case.context_lens, case.scale, case.H, case.Hk, case.d, case.B)
+    out = _run(c2)
+    assert torch.equal(out[0], out[1])
+    _assert_close(out, _oracle(oracle_mod, c2), torch.bfloat16, "shared prefix")
+
+
+# ---- combine, cache write, copy blocks ---------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_combine_matches_oracle(oracle_mod, d):
+    P = 64
+    lens = torch.tensor([1, 64, 65, 300, 0, 1000], dtype=torch.int32)
+    case = W.paged_case("comb", lens, 8, 2, d, 16, torch.float32, 92)
+    n_parts = int(math.ceil(int(lens.max()) / P))
+    po, pm, pl = oracle_mod.partials(case.q, case.k_cache, case.v_cache, case.block_tables, lens, P, n_parts)
+    po32, pm32, pl32 = po.float(), pm.float(), pl.float()
+    ref = oracle_mod.combine(po32, pm32, pl32)
+    got = api.pa_combine(po32.cuda(), pm32.cuda(), pl32.cuda(), lens.cuda(), P).cpu()
+    assert torch.isfinite(got).all()
+    assert (got.double() - ref).abs().max() < 1e-5
+    assert torch.count_nonzero(got[4]) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d,B", [(64, 8), (128, 16), (128, 32)])
+def test_cache_write_bit_exact(oracle_mod, dtype, d, B):
+    n_blocks, Hk, T = 40, 4, 75
+    g = W.generator(200 + d + B)
+    kc = W.randn(g, (n_blocks, Hk, B, d), dtype)
+    vc = W.randn(g, (n_blocks, Hk, B, d), dtype)
+    key = W.randn(g, (T, Hk, d), dtype)
+    val = W.randn(g, (T, Hk, d), dtype)
+    slots = torch.randperm(n_blocks * B, generator=g)[:T].to(torch.int64)
+    slots[::9] = -1
+    k_ref, v_ref = oracle_mod.cache_write(kc, vc, key, val, slots)
+    kd, vd = kc.cuda(), vc.cuda()
+    api.pa_cache_write(kd, vd, key.cuda(), val.cuda(), slots.cuda())
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(kd.cpu().view(bits), k_ref.view(bits))
+    assert torch.equal(vd.cpu().view(bits), v_ref.view(bits))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_copy_blocks_bit_exact(oracle_mod, dtype):
+    n_blocks, Hk, B, d = 64, 8, 16, 128
+    g = W.generator(300)
+    kc = W.randn(g, (n_blocks, Hk, B, d), dtype)
+    vc = W.randn(g, (n_blocks, Hk, B, d), dtype)
+    perm = torch.randperm(n_blocks, generator=g)
+    pairs = torch.stack([perm[:20], perm[20:40]], 1).to(torch.int32)  # distinct dsts, no dst is a src
+    k_ref, v_ref = oracle_mod.copy_blocks(kc, vc, pairs)
+    kd, vd = kc.cuda(), vc.cuda()
+    api.pa_copy_blocks(kd, vd, pairs.cuda())
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(kd.cpu().view(bits), k_ref.view(bits))
+    assert torch.equal(vd.cpu().view(bits), v_ref.view(bits))
