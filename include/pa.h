@@ -99,6 +99,32 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void
                     int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Paged decode attention that allocates nothing and takes no workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot call cudaMalloc: plugins
+ * whose host process owns the whole device-memory budget and forbids allocations by libraries,
+ * and serving loops that must not let an allocation (which can synchronise the device or fail
+ * under memory pressure) happen on the decode path.
+ *
+ * Arguments and results are those of pa_decode without `workspace` / `workspace_bytes`; the
+ * caller still passes every input and the output.  The workspace instead lives in one file-scope
+ * device array of 32 MiB (33554432 bytes) inside libpa, which every GPU that loads the library
+ * holds until the process exits.  Sizes whose pa_decode_workspace_size(...) exceeds 32 MiB are
+ * rejected with PA_ERR_INVALID_ARG and a message naming both sizes (a larger partition_size, or
+ * pa_decode with a caller-provided workspace, serves them).
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and caches it; make that first call before any stream capture.  Every
+ * call uses the same array, which keeps the last call's contents; the only fields that must
+ * start from known values (the unit counter, the unit count and the error word) are reset by the
+ * call's own first kernel.  Calls that overlap on the GPU (different streams, or different host
+ * threads on one device) race on the array: serialise them.  The error word of the array cannot
+ * be read through pa_workspace_error. */
+pa_status pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                            int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq,
+                            int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
+                            void* stream);
+
 /* Partition size (tokens) that pa_decode uses for these arguments when given 0. */
 int pa_decode_default_partition(int S, int Hk, int max_context_len);
 

@@ -25,6 +25,7 @@ SIGNATURES = {
     "pa_version": (ctypes.c_char_p, []),
     "pa_decode_workspace_size": (SZ, [I, I, I, I, I, I]),
     "pa_decode": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
+    "pa_decode_noalloc": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P]),
     "pa_decode_default_partition": (I, [I, I, I]),
     "pa_workspace_error": (I, [P, IP, P]),
     "pa_combine": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),

@@ -974,3 +974,56 @@ extern "C" pa_status pa_combine(void* out, pa_dtype out_dtype, const float* part
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_combine: launch failed: %s", cudaGetErrorString(e));
   return pa::ok();
 }
+
+// ---- decode without any device allocation --------------------------------------------------------
+// The decode workspace of pa_decode_noalloc lives in this file-scope device array instead of
+// caller memory.  Every GPU that loads the library holds it until the process exits.  In host
+// code `g_noalloc_scratch` only names a host-side stand-in, so its device address is fetched once
+// per device with cudaGetSymbolAddress (with that device current) and passed to the kernels.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       const int32_t* context_lens, int S, int H, int Hk, int d, int B,
+                                       int n_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                                       pa_dtype kv_dtype, int partition_size, void* stream) {
+  const size_t need = pa_decode_workspace_size(S, H, Hk, d, max_context_len, partition_size);
+  if (need == 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_noalloc: bad sizes");
+  if (need > kNoAllocScratchBytes)
+    return pa::fail(PA_ERR_INVALID_ARG,
+                    "pa_decode_noalloc: these sizes need %zu bytes of scratch; the built-in scratch holds %zu "
+                    "(use pa_decode with a caller-provided workspace, or a larger partition_size)",
+                    need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess)
+    return pa::fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+  return pa_decode(out, out_dtype, query, k_cache, v_cache, block_tables, context_lens, S, H, Hk, d, B, n_blocks,
+                   max_blocks_per_seq, max_context_len, scale, kv_dtype, partition_size, scratch,
+                   kNoAllocScratchBytes, stream);
+}
