@@ -52,6 +52,11 @@ WORKLOADS = {
     "mha13b_fp16": dict(S=64, H=40, Hk=40, d=128, B=16, dtype=torch.float16,
                         lens=lambda: W.lens_uniform(W.generator(2), 64, 1, 2048),
                         desc="13B-style MHA fp16: 64 seqs, 40 heads, d=128, B=16, context U[1,2048]"),
+    "shared_prefix_bf16": dict(S=128, H=32, Hk=8, d=128, B=16, dtype=torch.bfloat16, lens=None,
+                               desc="shared-prefix sampling and beam search, bf16: 32 requests x 4 sequences share "
+                                    "a 1024-token prompt (64 blocks at ref count 4), tails U[0,256]; every step "
+                                    "each sequence forks from a seeded parent among its request's 4, so shared "
+                                    "partial tail blocks are copied on write"),
     "long_bf16": dict(S=16, H=64, Hk=8, d=128, B=16, dtype=torch.bfloat16,
                       lens=lambda: W.lens_uniform(W.generator(5), 16, 16384, 32768),
                       desc="long-context bf16: 16 seqs, 64 q / 8 kv heads, d=128, B=16, context U[16384,32768]"),
@@ -66,9 +71,9 @@ class Workload:
         self.name, self.cfg = name, cfg
         self.S, self.H, self.Hk, self.d, self.B, self.dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
         self.es = torch.finfo(self.dtype).bits // 8
-        lens = cfg["lens"]().tolist()          # context length of each sequence after this step's token
+        lens = self._lengths()                 # context length of each sequence after this step's token
         B = self.B
-        need = sum(-(-c // B) for c in lens)
+        need = self._blocks_needed(lens)
         self.n_blocks = math.ceil(1.25 * need) + self.S * (growth_steps // B + 2)
         self.mgr = api.BlockManager(self.n_blocks, B)
         # Shuffle the free stack: take every block, release them in a seeded random order.
@@ -77,10 +82,7 @@ class Workload:
         for i in torch.randperm(self.n_blocks, generator=g).tolist():
             self.mgr.decref(blocks[i])
         self.seqs = torch.empty(self.S, dtype=torch.int32)
-        for i, c in enumerate(lens):
-            sid = self.mgr.seq_create()
-            self.mgr.reserve_slots(sid, c - 1)  # tokens cached before this step
-            self.seqs[i] = sid
+        self._make_sequences(lens)
         self.max_blocks = max(lens) // B + growth_steps // B + 4
         self.max_c = max(lens) + growth_steps + 1
         gen = torch.Generator(device=device).manual_seed(77 + seed_offset)
@@ -90,6 +92,28 @@ class Workload:
         self.device = device
         self.P = api.default_partition(self.S, self.Hk, self.max_c)
         self.workspace = api.alloc_workspace(self.S, self.H, self.Hk, self.d, self.max_c, self.P, device)
+
+    def _lengths(self):
+        return self.cfg["lens"]().tolist()
+
+    def _blocks_needed(self, lens):
+        return sum(-(-c // self.B) for c in lens)
+
+    def _make_sequences(self, lens):
+        for i, c in enumerate(lens):
+            sid = self.mgr.seq_create()
+            self.mgr.reserve_slots(sid, c - 1)  # tokens cached before this step
+            self.seqs[i] = sid
+
+    def trajectory(self, n_steps):
+        """Host block management for n_steps consecutive steps, uploaded to HBM."""
+        steps = []
+        for _ in range(n_steps):
+            slots, pairs, tables, lens = self.host_step()
+            dev = self.device
+            steps.append(dict(slots=slots.to(dev), pairs=pairs.to(dev), tables=tables.to(dev), lens=lens.to(dev),
+                              n_pairs=pairs.shape[0], lens_host=lens.tolist()))
+        return steps
 
     def host_step(self, slots=None, pairs=None, tables=None, lens=None):
         """One step of host block management: a slot per sequence, COW pairs, packed tables."""
@@ -105,6 +129,66 @@ class Workload:
         write = 2 * (S * Hk * d * es * 2) + 8 * S
         copy = n_pairs * 2 * (Hk * B * d * es) * 2
         return decode, decode + write + copy, kv
+
+
+class SharedPrefixWorkload(Workload):
+    """32 requests x 4 beams over a shared 1024-token prompt; beam-style forks every step."""
+
+    REQUESTS, WIDTH, PROMPT, TAIL_MAX = 32, 4, 1024, 256
+
+    def __init__(self, name, device, seed_offset=0, growth_steps=0):
+        self.rnd = torch.Generator().manual_seed(4 + seed_offset)
+        super().__init__(name, device, seed_offset, growth_steps + 64)
+
+    def _lengths(self):
+        tails = torch.randint(0, self.TAIL_MAX + 1, (self.REQUESTS * self.WIDTH,), generator=self.rnd)
+        self.tails = tails.tolist()
+        return [self.PROMPT + t + 1 for t in self.tails]
+
+    def _blocks_needed(self, lens):
+        B = self.B
+        prompt = self.REQUESTS * (self.PROMPT // B)
+        tails = sum(-(-(c - self.PROMPT) // B) + 1 for c in lens)
+        return prompt + 2 * tails
+
+    def _make_sequences(self, lens):
+        self.groups = []
+        i = 0
+        for r in range(self.REQUESTS):
+            root = self.mgr.seq_create()
+            self.mgr.reserve_slots(root, self.PROMPT)
+            beams = [root] + [self.mgr.seq_fork(root) for _ in range(self.WIDTH - 1)]
+            for b in beams:
+                self.mgr.reserve_slots(b, lens[i] - 1 - self.PROMPT)
+                self.seqs[i] = b
+                i += 1
+            self.groups.append(beams)
+
+    def host_step(self, slots=None, pairs=None, tables=None, lens=None):
+        # every beam picks a parent among its request's beams; children share the parent's blocks
+        i = 0
+        for r, beams in enumerate(self.groups):
+            parents = torch.randint(0, self.WIDTH, (self.WIDTH,), generator=self.rnd).tolist()
+            kids = [self.mgr.seq_fork(beams[p]) for p in parents]
+            for b in beams:
+                self.mgr.seq_free(b)
+            self.groups[r] = kids
+            for k in kids:
+                self.seqs[i] = k
+                i += 1
+        return super().host_step(slots, pairs, tables, lens)
+
+    def unique_kv_bytes(self, tables, lens):
+        used = set()
+        for s in range(self.S):
+            nb = -(-int(lens[s]) // self.B)
+            used.update(tables[s, :nb].tolist())
+        return len(used) * self.Hk * self.B * self.d * 2 * self.es
+
+
+def make_workload(name, device, seed_offset=0, growth_steps=0):
+    cls = SharedPrefixWorkload if name == "shared_prefix_bf16" else Workload
+    return cls(name, device, seed_offset, growth_steps)
 
 
 def load_peaks():
@@ -191,7 +275,8 @@ def run_pa(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     K, Wm = args.steps, args.warmup
     e2e_steps = min(K, args.e2e_steps)
-    wl = Workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + 2)
+    n_traj = 32 if args.workload == "shared_prefix_bf16" else 1
+    wl = make_workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + n_traj + 2)
     S, H, Hk, d = wl.S, wl.H, wl.Hk, wl.d
     gen = torch.Generator(device=dev).manual_seed(99 + rank)
     q = torch.randn((S, H, d), generator=gen, device=dev).to(wl.dtype)
@@ -199,50 +284,63 @@ def run_pa(args, rank, world, local_rank):
     val = torch.randn((S, Hk, d), generator=gen, device=dev).to(wl.dtype)
     out = torch.empty((S, H, d), dtype=wl.dtype, device=dev)
 
-    # The step whose inputs sit in HBM for the device-timed loop.
-    slots, pairs, tables, lens = wl.host_step()
-    d_slots, d_pairs = slots.to(dev), pairs.to(dev)
-    d_tables, d_lens = tables.to(dev), lens.to(dev)
-    n_pairs = pairs.shape[0]
-    decode_bytes, step_bytes, kv_bytes = wl.step_bytes(lens.tolist(), n_pairs)
+    # Host block management for a fixed trajectory of steps, done before timing; the timed loop
+    # replays it with every input in HBM (one step for the decode-only workloads).
+    traj = wl.trajectory(n_traj)
+    for st in traj:
+        st["decode_bytes"], st["step_bytes"], st["kv_bytes"] = wl.step_bytes(st["lens_host"], st["n_pairs"])
     max_parts = -(-wl.max_c // wl.P)
-    launches_per_step = 2 + (1 if max_parts > 1 else 0) + 1 + (1 if n_pairs else 0)
+    launches = [2 + (1 if max_parts > 1 else 0) + 1 + (1 if st["n_pairs"] else 0) for st in traj]
 
-    def device_step(ev0=None, ev1=None):
-        if n_pairs:
-            api.pa_copy_blocks(wl.k_cache, wl.v_cache, d_pairs)
-        api.pa_cache_write(wl.k_cache, wl.v_cache, key, val, d_slots)
-        if ev0 is not None:
-            ev0.record()
-        api.pa_decode(q, wl.k_cache, wl.v_cache, d_tables, d_lens, max_context_len=wl.max_c, out=out,
+    def device_step(st, evs=None):
+        if evs is not None:
+            evs[0].record()
+        if st["n_pairs"]:
+            api.pa_copy_blocks(wl.k_cache, wl.v_cache, st["pairs"])
+        if evs is not None:
+            evs[1].record()
+        api.pa_cache_write(wl.k_cache, wl.v_cache, key, val, st["slots"])
+        if evs is not None:
+            evs[2].record()
+        api.pa_decode(q, wl.k_cache, wl.v_cache, st["tables"], st["lens"], max_context_len=wl.max_c, out=out,
                       partition_size=wl.P, workspace=wl.workspace)
-        if ev1 is not None:
-            ev1.record()
+        if evs is not None:
+            evs[3].record()
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
     clocks = ClockSampler(local_rank)
-    for _ in range(Wm):
-        device_step()
+    for i in range(Wm):
+        device_step(traj[i % n_traj])
     torch.cuda.synchronize()
     assert api.workspace_error(wl.workspace) == 0, "decode reported an error"
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record()
     for i in range(K):
-        device_step(*evs[i])
+        device_step(traj[i % n_traj], evs[i])
     stop.record()
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
     clocks.mark(t_wall0, t_wall1)
     total_ms = start.elapsed_time(stop)
-    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    copy_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    write_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    step_bytes = statistics.mean(traj[i % n_traj]["step_bytes"] for i in range(K))
+    decode_bytes = statistics.mean(traj[i % n_traj]["decode_bytes"] for i in range(K))
+    kv_bytes = statistics.mean(traj[i % n_traj]["kv_bytes"] for i in range(K))
+    copy_bytes = statistics.mean(traj[i % n_traj]["n_pairs"] * 2 * Hk * wl.B * d * wl.es * 2 for i in range(K))
+    write_bytes = 2 * (S * Hk * d * wl.es * 2) + 8 * S
+    n_pairs = statistics.mean(st["n_pairs"] for st in traj)
+    lens = traj[0]["lens"].cpu()
+    launches_total = sum(launches[i % n_traj] for i in range(K))
 
     # ---- end to end through the API, from pinned host memory ----
     pin = lambda t: t.cpu().pin_memory()
@@ -333,9 +431,16 @@ def run_pa(args, rank, world, local_rank):
             "partition_size": wl.P,
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush",
             "step": "host block manager -> pa_copy_blocks -> pa_cache_write -> pa_decode (plan, decode, combine)",
-            "step_bytes": step_bytes,
+            "step_bytes": round(step_bytes),
             "cow_pairs_per_step": n_pairs,
+            "trajectory_steps": n_traj,
+            **({"unique_kv_bytes_step0": wl.unique_kv_bytes(traj[0]["tables"].cpu(), lens),
+                "logical_kv_bytes_step0": traj[0]["kv_bytes"]} if hasattr(wl, "unique_kv_bytes") else {}),
         },
+        "kernel_ms": {"copy_blocks": round(copy_ms, 5), "cache_write": round(write_ms, 5),
+                      "decode": round(decode_ms, 5)},
+        "kernel_gbs": {"copy_blocks": round(copy_bytes / (copy_ms * 1e-3) / 1e9, 2) if copy_bytes else None,
+                       "cache_write": round(write_bytes / (write_ms * 1e-3) / 1e9, 2)},
         "seqs_per_s": round(S * world / (ms_per_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
         "roofline": {
@@ -360,7 +465,7 @@ def run_pa(args, rank, world, local_rank):
             "ms_per_step": round(e2e_ms / e2e_steps, 5),
             "note": "host block manager + H2D of the step's inputs + kernels + D2H of o, synchronised each step",
         },
-        "gpu_launches": K * launches_per_step,
+        "gpu_launches": launches_total,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, lens.tolist(), q, target_s=args.cpu_seconds)

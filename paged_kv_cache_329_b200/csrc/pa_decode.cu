@@ -30,6 +30,8 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "pa_device.cuh"
@@ -268,7 +270,267 @@ __device__ __forceinline__ void write_rows(OutT* base, const float (&acc)[G][AC]
     }
 }
 
-template <class T, int D, int G>
+
+// ---- tensor-core consumers (16-bit caches) ---------------------------------------------------------
+// Each consumer warp owns 16 token rows of every 64-token tile.  With tokens in M and the head group
+// in N (g <= 8 heads, zero-padded to 8):
+//   S^T[16 tok x 8 heads]  = K[16 tok x d] * Q^T[d x 8]          (d/16 mma.m16n8k16, K by ldmatrix)
+//   O^T[d x 8 heads]      += V^T[d x 16 tok] * P^T[16 tok x 8]   (d/16 m-tiles, V by ldmatrix.trans)
+// P^T comes from the S^T accumulator layout by an 8x8 register transpose (movmatrix) and is fed as a
+// 16-bit pair hi + lo (hi = p rounded, lo = p - hi rounded), so the weights keep ~16 bits of
+// precision; scores, maxima, sums and the output accumulate in fp32.  Tokens past the sequence's
+// length get score -inf and their V elements are zeroed in registers (the shared tile may hold
+// stale data or unused slots there).
+template <class T, int D, int G, class C>
+__device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, StageMeta* meta, uint64_t* full,
+                                            uint64_t* empty, uint64_t* epi, float* ml, float* merge,
+                                            const DecodeArgs& a, int warp, int lane) {
+  using M = pa::Mma<T>;
+  constexpr int KS = D / 16;  // k-steps of q.k and m-tiles of p.V
+  constexpr int NF4 = G * D / 4;
+  constexpr int NMINE = (NF4 + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
+  const int gq = lane >> 2, tq = lane & 3;  // mma groupID / thread-in-group
+  const int tid = warp * 32 + lane;
+  uint32_t bq[KS][2];
+  float acc[KS][4];
+  float m_run[2], l_run[2];
+#pragma unroll
+  for (int k = 0; k < KS; ++k) {
+    bq[k][0] = bq[k][1] = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
+  }
+  m_run[0] = m_run[1] = -INFINITY;
+  l_run[0] = l_run[1] = 0.f;
+
+  int stage = 0;
+  uint32_t phase = 0, epi_phase = 0;
+  auto epi_sync = [&]() -> bool {
+    pa::mbar_arrive(epi);
+    const bool done = pa::mbar_wait(epi, epi_phase);
+    epi_phase ^= 1;
+    if (!done && lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    return done;
+  };
+  // ldmatrix row/chunk assignment of this lane (tile index = lane / 8)
+  const int ld_row = ((lane >> 3) & 1) * 8 + (lane & 7);      // q.k: tiles (tok 0-7, tok 8-15) x (lo, hi dims)
+  const int ld_hi = lane >> 4;
+  const int ldt_row = (lane >> 4) * 8 + (lane & 7);            // p.V: tiles (lo, hi dims) x (tok 0-7, tok 8-15)
+  const int ldt_hi = (lane >> 3) & 1;
+
+  while (true) {
+    if (!pa::mbar_wait(&full[stage], phase)) {
+      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      return;
+    }
+    const StageMeta mt = meta[stage];
+    if (mt.flags & kDone) break;
+    const uint8_t* ks = stages + stage * C::kStageBytes;
+    const uint8_t* vs = ks + C::kKVBytes;
+    const int ntok = mt.ntok;
+
+    if (mt.flags & kFirst) {
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qslots + stage * C::kQSlot);
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        bq[k][0] = gq < G ? q32[(gq * D + k * 16 + 2 * tq) >> 1] : 0u;
+        bq[k][1] = gq < G ? q32[(gq * D + k * 16 + 8 + 2 * tq) >> 1] : 0u;
+      }
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
+    }
+
+    const int r0 = warp * 16;
+    if (r0 < ntok) {
+      // ---- scores S^T = K Q^T ----
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t kbase = pa::smem_addr(ks);
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        const int row = r0 + ld_row, c = 2 * k + ld_hi;
+        uint32_t af[4];
+        pa::ldsm_x4(af, kbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+        M::run(sacc, af, bq[k]);
+      }
+      // ---- online softmax; this lane holds tokens gq, gq+8 for heads 2tq, 2tq+1 ----
+      const bool v0 = r0 + gq < ntok, v1 = r0 + gq + 8 < ntok;
+      float x[4];
+      x[0] = v0 ? sacc[0] * a.scale_log2 : -INFINITY;
+      x[1] = v0 ? sacc[1] * a.scale_log2 : -INFINITY;
+      x[2] = v1 ? sacc[2] * a.scale_log2 : -INFINITY;
+      x[3] = v1 ? sacc[3] * a.scale_log2 : -INFINITY;
+      float mx[2] = {fmaxf(x[0], x[2]), fmaxf(x[1], x[3])};
+#pragma unroll
+      for (int msk = 4; msk <= 16; msk <<= 1) {
+        mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], msk));
+        mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], msk));
+      }
+      float alpha[2], mn[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        mn[j] = fmaxf(m_run[j], mx[j]);
+        alpha[j] = (mn[j] == -INFINITY) ? 1.f : exp2f(m_run[j] - mn[j]);
+        m_run[j] = mn[j];
+      }
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = (mn[e & 1] == -INFINITY) ? 0.f : exp2f(x[e] - mn[e & 1]);
+      l_run[0] = l_run[0] * alpha[0] + (p[0] + p[2]);
+      l_run[1] = l_run[1] * alpha[1] + (p[1] + p[3]);
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        acc[k][0] *= alpha[0];
+        acc[k][1] *= alpha[1];
+        acc[k][2] *= alpha[0];
+        acc[k][3] *= alpha[1];
+      }
+      // ---- P^T fragments (hi and lo parts) ----
+      float r[4];
+      const uint32_t h01 = M::pack(p[0], p[1], r[0], r[1]);
+      const uint32_t h23 = M::pack(p[2], p[3], r[2], r[3]);
+      float dummy0, dummy1;
+      const uint32_t l01 = M::pack(p[0] - r[0], p[1] - r[1], dummy0, dummy1);
+      const uint32_t l23 = M::pack(p[2] - r[2], p[3] - r[3], dummy0, dummy1);
+      const uint32_t bh[2] = {pa::movmatrix_trans(h01), pa::movmatrix_trans(h23)};
+      const uint32_t bl[2] = {pa::movmatrix_trans(l01), pa::movmatrix_trans(l23)};
+      // ---- O^T += V^T P^T ----
+      const bool partial = r0 + 16 > ntok;
+      uint32_t mask01 = 0xffffffffu, mask23 = 0xffffffffu;
+      if (partial) {
+        const int t0 = r0 + 2 * tq;
+        mask01 = (t0 < ntok ? 0x0000ffffu : 0u) | (t0 + 1 < ntok ? 0xffff0000u : 0u);
+        mask23 = (t0 + 8 < ntok ? 0x0000ffffu : 0u) | (t0 + 9 < ntok ? 0xffff0000u : 0u);
+      }
+      const uint32_t vbase = pa::smem_addr(vs);
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        const int row = r0 + ldt_row, c = 2 * k + ldt_hi;
+        uint32_t af[4];
+        pa::ldsm_x4_trans(af, vbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+        af[0] &= mask01;
+        af[1] &= mask01;
+        af[2] &= mask23;
+        af[3] &= mask23;
+        M::run(acc[k], af, bh);
+        M::run(acc[k], af, bl);
+      }
+    }
+
+    __syncwarp();
+    if (lane == 0) pa::mbar_arrive(&empty[stage]);
+
+    if (mt.flags & kLast) {
+      // ---- merge the four warps in a fixed order: (w0 + w2) + (w1 + w3) ----
+      float lsum[2] = {l_run[0], l_run[1]};
+#pragma unroll
+      for (int msk = 4; msk <= 16; msk <<= 1) {
+        lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], msk);
+        lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], msk);
+      }
+      if (gq == 0) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          if (2 * tq + j < G) {
+            ml[(warp * G + 2 * tq + j) * 2] = m_run[j];
+            ml[(warp * G + 2 * tq + j) * 2 + 1] = lsum[j];
+          }
+      }
+      if (!epi_sync()) return;
+      // weights of this warp's heads, and 1/den (or M, den) for the heads this thread writes out
+      float wmine[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int h = 2 * tq + j;
+        wmine[j] = 0.f;
+        if (h < G) {
+          float mxh = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) mxh = fmaxf(mxh, ml[(w * G + h) * 2]);
+          wmine[j] = (m_run[j] == -INFINITY) ? 0.f : exp2f(m_run[j] - mxh);
+        }
+      }
+      float outM[NMINE], outDen[NMINE];
+#pragma unroll
+      for (int i = 0; i < NMINE; ++i) {
+        const int f = tid + i * kConsumerWarps * 32;
+        const int h = f < NF4 ? (f * 4) / D : 0;
+        float mxh = -INFINITY, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mxh = fmaxf(mxh, ml[(w * G + h) * 2]);
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = ml[(w * G + h) * 2];
+          if (mw != -INFINITY) den += exp2f(mw - mxh) * ml[(w * G + h) * 2 + 1];
+        }
+        outM[i] = mxh;
+        outDen[i] = den;
+      }
+      // this thread's accumulator elements: dims 16k + gq (+8), heads 2tq, 2tq+1
+      auto put = [&](float* buf, bool add) {
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = 2 * tq + (e & 1);
+            if (h < G) {
+              float* dst = buf + h * D + 16 * k + gq + (e >> 1) * 8;
+              *dst = add ? *dst + acc[k][e] * wmine[e & 1] : acc[k][e] * wmine[e & 1];
+            }
+          }
+      };
+      if (warp >= 2) put(merge + (warp - 2) * G * D, false);
+      if (!epi_sync()) return;
+      if (warp < 2) put(merge + warp * G * D, true);
+      if (!epi_sync()) return;
+      const size_t row = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;
+#pragma unroll
+      for (int i = 0; i < NMINE; ++i) {
+        const int f = tid + i * kConsumerWarps * 32;
+        if (f < NF4) {
+          const int h = (f * 4) / D, dd = (f * 4) % D;
+          const float4 x0 = *reinterpret_cast<const float4*>(merge + f * 4);
+          const float4 x1 = *reinterpret_cast<const float4*>(merge + G * D + f * 4);
+          float v[4] = {x0.x + x1.x, x0.y + x1.y, x0.z + x1.z, x0.w + x1.w};
+          if (mt.flags & kSingle) {
+            const float inv = outDen[i] > 0.f ? 1.f / outDen[i] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] *= inv;
+            if (a.out_dtype == PA_F32)
+              pa::store_floats<float, 4>(static_cast<float*>(a.out) + (row + h) * D + dd, v);
+            else if (a.out_dtype == PA_F16)
+              pa::store_floats<__half, 4>(static_cast<__half*>(a.out) + (row + h) * D + dd, v);
+            else
+              pa::store_floats<__nv_bfloat16, 4>(static_cast<__nv_bfloat16*>(a.out) + (row + h) * D + dd, v);
+          } else {
+            const size_t pidx = (row + h) * a.max_parts + mt.part;
+            pa::store_floats<float, 4>(a.part_o + pidx * D + dd, v);
+            if (dd == 0) {
+              a.part_m[pidx] = outM[i] == -INFINITY ? -INFINITY : outM[i] * kLn2;
+              a.part_l[pidx] = outDen[i];
+            }
+          }
+        }
+      }
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
+    }
+
+    if (++stage == C::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+}
+
+template <class T, int D, int G, bool kMma>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const DecodeArgs a) {
@@ -393,6 +655,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   }
 
   // ================================== consumer warps ============================================
+  if constexpr (kMma) {
+    consume_mma<T, D, G, C>(stages, qslots, meta, full, empty, epi, ml, merge, a, warp, lane);
+  } else {
   const int grp = lane / L, l = lane % L;
   const int my_tok = token_of_lane<L, R>(l);
   const bool primary = primary_lane<L, R>(l);
@@ -679,6 +944,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       phase ^= 1;
     }
   }
+  }  // consumers
 }
 
 // ---- log-sum-exp combine -----------------------------------------------------------------------
@@ -802,17 +1068,17 @@ DeviceInfo device_info() {
   return di;
 }
 
-template <class T, int D, int G>
+template <class T, int D, int G, bool kMma>
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int max_units,
                           cudaStream_t st) {
   using C = Cfg<T, D, G>;
   static int occupancy = -1;  // per instantiation; device properties are uniform on a B200 node
   cudaError_t e = cudaSuccess;
   if (occupancy < 0) {
-    e = cudaFuncSetAttribute(decode_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(decode_kernel<T, D, G, kMma>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<T, D, G>, kThreads, C::kSmemBytes);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<T, D, G, kMma>, kThreads, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     occupancy = occ < 1 ? 1 : occ;
   }
@@ -820,25 +1086,40 @@ cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const De
   long long grid = static_cast<long long>(di.sms) * occupancy;
   if (grid > max_units) grid = max_units;
   if (grid < 1) grid = 1;
-  decode_kernel<T, D, G><<<static_cast<int>(grid), kThreads, C::kSmemBytes, st>>>(tk, tv, a);
+  decode_kernel<T, D, G, kMma><<<static_cast<int>(grid), kThreads, C::kSmemBytes, st>>>(tk, tv, a);
   return cudaGetLastError();
 }
 
-template <class T, int D>
+// Tensor-core consumers for 16-bit caches unless PA_DECODE_CONSUMER=cuda_core; fp32 caches always
+// use the CUDA-core consumers.
+bool use_tensor_cores() {
+  const char* v = std::getenv("PA_DECODE_CONSUMER");
+  return !(v && std::strcmp(v, "cuda_core") == 0);
+}
+
+template <class T, int D, bool kMma>
 cudaError_t dispatch_g(int g, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int max_units,
                        cudaStream_t st) {
   switch (g) {
-    case 1: return launch_decode<T, D, 1>(tk, tv, a, max_units, st);
-    case 2: return launch_decode<T, D, 2>(tk, tv, a, max_units, st);
-    case 4: return launch_decode<T, D, 4>(tk, tv, a, max_units, st);
-    default: return launch_decode<T, D, 8>(tk, tv, a, max_units, st);
+    case 1: return launch_decode<T, D, 1, kMma>(tk, tv, a, max_units, st);
+    case 2: return launch_decode<T, D, 2, kMma>(tk, tv, a, max_units, st);
+    case 4: return launch_decode<T, D, 4, kMma>(tk, tv, a, max_units, st);
+    default: return launch_decode<T, D, 8, kMma>(tk, tv, a, max_units, st);
   }
 }
 
-template <class T>
+template <class T, bool kMma>
 cudaError_t dispatch_d(int d, int g, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
                        int max_units, cudaStream_t st) {
-  return d == 64 ? dispatch_g<T, 64>(g, tk, tv, a, max_units, st) : dispatch_g<T, 128>(g, tk, tv, a, max_units, st);
+  return d == 64 ? dispatch_g<T, 64, kMma>(g, tk, tv, a, max_units, st)
+                 : dispatch_g<T, 128, kMma>(g, tk, tv, a, max_units, st);
+}
+
+template <class T>
+cudaError_t dispatch_16bit(int d, int g, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a,
+                           int max_units, cudaStream_t st) {
+  return use_tensor_cores() ? dispatch_d<T, true>(d, g, tk, tv, a, max_units, st)
+                            : dispatch_d<T, false>(d, g, tk, tv, a, max_units, st);
 }
 
 int default_partition(int S, int Hk, int max_context_len) {
@@ -944,9 +1225,9 @@ extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query,
 
   const long long units = static_cast<long long>(S) * Hk * max_parts;
   const int max_units = static_cast<int>(units < (1ll << 30) ? units : (1ll << 30));
-  if (kv_dtype == PA_F32) e = dispatch_d<float>(d, g, tk, tv, a, max_units, st);
-  else if (kv_dtype == PA_F16) e = dispatch_d<__half>(d, g, tk, tv, a, max_units, st);
-  else e = dispatch_d<__nv_bfloat16>(d, g, tk, tv, a, max_units, st);
+  if (kv_dtype == PA_F32) e = dispatch_d<float, false>(d, g, tk, tv, a, max_units, st);
+  else if (kv_dtype == PA_F16) e = dispatch_16bit<__half>(d, g, tk, tv, a, max_units, st);
+  else e = dispatch_16bit<__nv_bfloat16>(d, g, tk, tv, a, max_units, st);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s", cudaGetErrorString(e));
 
   if (max_parts > 1) {

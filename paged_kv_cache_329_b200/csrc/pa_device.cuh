@@ -102,6 +102,72 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
   return v;
 }
 
+// ---- warp-level tensor-core helpers (mma.sync m16n8k16, fp32 accumulate) ------------------------
+
+// Four 8x8 tiles of 16-bit elements; lane L supplies the address of row L%8 of tile L/8.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// As ldsm_x4, each 8x8 tile transposed on the way into registers.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Transposes an 8x8 tile of 16-bit elements held one pair per lane (row L/4, columns 2(L%4)..+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+template <class T>
+struct Mma;
+
+template <>
+struct Mma<__nv_bfloat16> {
+  // d[16x8] += a[16x16] (row-major) * b[16x8] (column-major), bf16 inputs, fp32 accumulators.
+  __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  }
+  // Packs two floats (x0 in the low half) rounded to nearest even; returns the rounded values too.
+  __device__ __forceinline__ static uint32_t pack(float x0, float x1, float& r0, float& r1) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(x0, x1);
+    r0 = __low2float(v);
+    r1 = __high2float(v);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+};
+
+template <>
+struct Mma<__half> {
+  __device__ __forceinline__ static void run(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+  }
+  __device__ __forceinline__ static uint32_t pack(float x0, float x1, float& r0, float& r1) {
+    const __half2 v = __floats2half2_rn(x0, x1);
+    r0 = __low2float(v);
+    r1 = __high2float(v);
+    return *reinterpret_cast<const uint32_t*>(&v);
+  }
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---- 16-byte chunk -> floats -------------------------------------------------------------------
 
 template <class T>

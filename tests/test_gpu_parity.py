@@ -18,6 +18,13 @@ pytestmark = pytest.mark.gpu
 TOL = {torch.float32: 1e-5, torch.float16: 2e-3, torch.bfloat16: 2e-3}
 
 
+@pytest.fixture(params=["mma", "cuda_core"])
+def consumer(request, monkeypatch):
+    """16-bit caches: tensor-core consumers (default) or CUDA-core consumers."""
+    monkeypatch.setenv("PA_DECODE_CONSUMER", request.param)
+    return request.param
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _lib():
     from paged_kv_cache_329_b200 import build
@@ -79,7 +86,7 @@ def test_tiny_fp32(oracle_mod):
     _assert_close(_run(case), ref, torch.float32, "tiny_fp32")
 
 
-def test_mha13b_fp16_with_cache_write(oracle_mod):
+def test_mha13b_fp16_with_cache_write(oracle_mod, consumer):
     case = W.mha13b_fp16()
     tables, lens, slots = W.new_token_slots(case, W.generator(102))
     g = W.generator(103)
@@ -99,7 +106,7 @@ def test_mha13b_fp16_with_cache_write(oracle_mod):
     _assert_ulp(_run(dev2, torch.float16, max_c=int(lens.max())), ref, "mha13b_fp16 fp16 out")
 
 
-def test_gqa8k_bf16_full_size_sampled(oracle_mod):
+def test_gqa8k_bf16_full_size_sampled(oracle_mod, consumer):
     case = W.gqa8k_bf16(device="cuda")
     lens = case.context_lens.cpu()
     order = torch.argsort(lens)
@@ -112,7 +119,7 @@ def test_gqa8k_bf16_full_size_sampled(oracle_mod):
 
 
 @pytest.mark.parametrize("B", [8, 16, 32])
-def test_long_context_full_size_sampled(oracle_mod, B):
+def test_long_context_full_size_sampled(oracle_mod, B, consumer):
     case = W.long_bf16(B=B, device="cuda")
     sample = [0, 7, int(torch.argmax(case.context_lens.cpu()))]
     ref = _oracle(oracle_mod, case, sample)
@@ -130,7 +137,9 @@ EDGE_LENS = [1, 7, 8, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 255, 256, 25
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("B", [8, 16, 32])
-def test_edge_lengths(oracle_mod, dtype, g, d, B):
+def test_edge_lengths(oracle_mod, dtype, g, d, B, consumer):
+    if dtype == torch.float32 and consumer == "cuda_core":
+        pytest.skip("fp32 caches always use the CUDA-core consumers")
     Hk = 2
     case = W.paged_case("edge", EDGE_LENS, g * Hk, Hk, d, B, dtype, 1000 + g * 7 + d + B)
     ref = _oracle(oracle_mod, case)
@@ -138,7 +147,7 @@ def test_edge_lengths(oracle_mod, dtype, g, d, B):
         _assert_close(_run(case, P=P), ref, dtype, f"{dtype} g={g} d={d} B={B} P={P}")
 
 
-def test_zero_length_sequences_give_zero(oracle_mod):
+def test_zero_length_sequences_give_zero(oracle_mod, consumer):
     case = W.paged_case("zero", [0, 5, 0, 300, 0], 8, 2, 128, 16, torch.bfloat16, 77)
     out = _run(case, P=64)
     assert torch.count_nonzero(out[0]) == 0 and torch.count_nonzero(out[2]) == 0 and torch.count_nonzero(out[4]) == 0
@@ -150,7 +159,7 @@ def test_all_empty_batch():
     assert torch.count_nonzero(_run(case)) == 0
 
 
-def test_output_types(oracle_mod):
+def test_output_types(oracle_mod, consumer):
     case = W.paged_case("types", [3, 70, 600], 16, 4, 128, 16, torch.float16, 79)
     ref = _oracle(oracle_mod, case)
     _assert_close(_run(case, torch.float32), ref, torch.float16, "f32 out")
@@ -161,7 +170,7 @@ def test_output_types(oracle_mod):
 # ---- determinism and placement -----------------------------------------------------------------
 
 @pytest.mark.parametrize("B", [8, 16, 32])
-def test_physical_permutation_is_bit_identical(B):
+def test_physical_permutation_is_bit_identical(B, consumer):
     case = W.paged_case("perm", [1, B + 1, 200, 700, 1500], 32, 8, 128, B, torch.bfloat16, 80 + B, pool_factor=2.0)
     o1 = _run(case, P=256)
     n = case.n_blocks
@@ -179,7 +188,7 @@ def test_physical_permutation_is_bit_identical(B):
     assert torch.equal(o1, _run(case, P=256))  # and a repeat call
 
 
-def test_split_and_unsplit_agree(oracle_mod):
+def test_split_and_unsplit_agree(oracle_mod, consumer):
     case = W.paged_case("split", [2000, 3000, 64, 4097], 32, 8, 128, 16, torch.bfloat16, 90)
     ref = _oracle(oracle_mod, case)
     outs = [_run(case, P=P) for P in (64, 512, 4160)]   # 4160 >= every length: no split at all
@@ -188,7 +197,7 @@ def test_split_and_unsplit_agree(oracle_mod):
     assert (outs[0] - outs[2]).abs().max() < 1e-4
 
 
-def test_shared_prefix_reads_same_blocks(oracle_mod):
+def test_shared_prefix_reads_same_blocks(oracle_mod, consumer):
     # Sequences whose tables share the prompt blocks and whose tails and queries match produce
     # identical outputs.
     case = W.paged_case("pref", [1030, 1030], 32, 8, 128, 16, torch.bfloat16, 91, sentinel="none", n_blocks=200)
