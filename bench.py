@@ -268,6 +268,19 @@ class ClockSampler:
                 "samples": len(sms)}
 
 
+def reduce_max(values, world, device="cpu"):
+    """Element-wise maximum over ranks (every rank gets it); the slowest rank sets the time."""
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_value(bytes_per_rank_step, steps, world, max_ms):
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
+
+
 # ---- the GPU arm ----------------------------------------------------------------------------------
 
 def run_pa(args, rank, world, local_rank):
@@ -398,16 +411,13 @@ def run_pa(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
     clock_info = clocks.finish()
 
-    # max over ranks
-    t = torch.tensor([total_ms, e2e_ms, decode_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms, decode_ms = t.tolist()
+    total_ms, e2e_ms, decode_ms, copy_ms, write_ms = reduce_max([total_ms, e2e_ms, decode_ms, copy_ms, write_ms],
+                                                                world, dev)
     if rank != 0:
         return None
 
     peak, peak_kind = load_peaks()
-    value = world * step_bytes * K / (total_ms * 1e-3) / 1e9
+    value = aggregate_value(step_bytes, K, world, total_ms)
     achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
     ms_per_step = total_ms / K
     line = {

@@ -42,11 +42,7 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
-def _load():
-    global _lib
-    if _lib is not None:
-        return _lib
-    lib = ctypes.CDLL(build())
+def _declare(lib):
     P, I, D, L = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_long
     lib.oracle_decode.argtypes = [P, P, I, P, P, I, P, P, I, I, I, I, I, I, I, D, I]
     lib.oracle_decode.restype = I
@@ -64,8 +60,39 @@ def _load():
     lib.oracle_hardware_threads.restype = I
     lib.oracle_elem_to_double.argtypes = [P, I, L]
     lib.oracle_elem_to_double.restype = D
-    _lib = lib
     return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+_active = None  # a library other than liboracle.so while `variant(...)` is in effect
+
+
+def _L():
+    return _active if _active is not None else _load()
+
+
+class variant:
+    """Context manager: route every function of this module to another build of oracle.cpp
+    (used by the tests that check the pins catch planted mistakes)."""
+
+    def __init__(self, so_path: str):
+        self.lib = _declare(ctypes.CDLL(so_path))
+
+    def __enter__(self):
+        global _active
+        self._prev, _active = _active, self.lib
+        return self
+
+    def __exit__(self, *exc):
+        global _active
+        _active = self._prev
+        return False
 
 
 def _cpu(t: torch.Tensor) -> torch.Tensor:
@@ -81,12 +108,12 @@ def _code(t: torch.Tensor) -> int:
 
 
 def hardware_threads() -> int:
-    return _load().oracle_hardware_threads()
+    return _L().oracle_hardware_threads()
 
 
 def elem_to_double(t: torch.Tensor, idx: int) -> float:
     t = _cpu(t)
-    return _load().oracle_elem_to_double(t.data_ptr(), _code(t), idx)
+    return _L().oracle_elem_to_double(t.data_ptr(), _code(t), idx)
 
 
 def _shape(q, k_cache, block_tables):
@@ -105,7 +132,7 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale=None, n_thread
     if scale is None:
         scale = 1.0 / d ** 0.5
     out = torch.empty((S, H, d), dtype=torch.float64)
-    rc = _load().oracle_decode(
+    rc = _L().oracle_decode(
         out.data_ptr(), q.data_ptr(), _code(q), k_cache.data_ptr(), v_cache.data_ptr(), _code(k_cache),
         bt.data_ptr(), cl.data_ptr(), S, H, Hk, d, B, n_blocks, mb, float(scale), int(n_threads),
     )
@@ -122,7 +149,7 @@ def decode_blockwise(q, k_cache, v_cache, block_tables, context_lens, scale=None
     if scale is None:
         scale = 1.0 / d ** 0.5
     out = torch.empty((S, H, d), dtype=torch.float64)
-    rc = _load().oracle_decode_blockwise(
+    rc = _L().oracle_decode_blockwise(
         out.data_ptr(), q.data_ptr(), _code(q), k_cache.data_ptr(), v_cache.data_ptr(), _code(k_cache),
         bt.data_ptr(), cl.data_ptr(), S, H, Hk, d, B, n_blocks, mb, float(scale),
     )
@@ -141,7 +168,7 @@ def partials(q, k_cache, v_cache, block_tables, context_lens, partition_size, n_
     po = torch.empty((S, H, n_parts, d), dtype=torch.float64)
     pm = torch.empty((S, H, n_parts), dtype=torch.float64)
     pl = torch.empty((S, H, n_parts), dtype=torch.float64)
-    rc = _load().oracle_partials(
+    rc = _L().oracle_partials(
         po.data_ptr(), pm.data_ptr(), pl.data_ptr(), n_parts, partition_size, q.data_ptr(), _code(q),
         k_cache.data_ptr(), v_cache.data_ptr(), _code(k_cache), bt.data_ptr(), cl.data_ptr(),
         S, H, Hk, d, B, n_blocks, mb, float(scale),
@@ -158,7 +185,7 @@ def combine(part_o, part_m, part_l):
     want = torch.float32 if f32 else torch.float64
     po, pm, pl = (_cpu(t.to(want)) for t in (part_o, part_m, part_l))
     out = torch.empty((S, H, d), dtype=torch.float64)
-    _load().oracle_combine(out.data_ptr(), po.data_ptr(), pm.data_ptr(), pl.data_ptr(), int(f32), S, H, n_parts, d)
+    _L().oracle_combine(out.data_ptr(), po.data_ptr(), pm.data_ptr(), pl.data_ptr(), int(f32), S, H, n_parts, d)
     return out
 
 
@@ -168,7 +195,7 @@ def cache_write(k_cache, v_cache, key, value, slot_mapping):
     key, value = _cpu(key.to(kc.dtype)), _cpu(value.to(kc.dtype))
     sm = _cpu(slot_mapping.to(torch.int64))
     n_blocks, Hk, B, d = kc.shape
-    rc = _load().oracle_cache_write(
+    rc = _L().oracle_cache_write(
         kc.data_ptr(), vc.data_ptr(), key.data_ptr(), value.data_ptr(), sm.data_ptr(),
         key.shape[0], Hk, d, B, n_blocks, _code(kc),
     )
@@ -182,7 +209,7 @@ def copy_blocks(k_cache, v_cache, pairs):
     kc, vc = _cpu(k_cache).clone(), _cpu(v_cache).clone()
     pr = _cpu(pairs.to(torch.int32).reshape(-1, 2))
     n_blocks, Hk, B, d = kc.shape
-    rc = _load().oracle_copy_blocks(kc.data_ptr(), vc.data_ptr(), pr.data_ptr(), pr.shape[0], Hk, d, B, n_blocks, _code(kc))
+    rc = _L().oracle_copy_blocks(kc.data_ptr(), vc.data_ptr(), pr.data_ptr(), pr.shape[0], Hk, d, B, n_blocks, _code(kc))
     if rc != 0:
         raise ValueError("oracle_copy_blocks: block id out of range")
     return kc, vc
