@@ -66,7 +66,7 @@ WORKLOADS = {
 class Workload:
     """Sequences in a native block manager over a shuffled pool, random K/V in HBM."""
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0):
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0):
         cfg = WORKLOADS[name]
         self.name, self.cfg = name, cfg
         self.S, self.H, self.Hk, self.d, self.B, self.dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
@@ -90,7 +90,7 @@ class Workload:
         self.k_cache = torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(self.dtype)
         self.v_cache = torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(self.dtype)
         self.device = device
-        self.P = api.default_partition(self.S, self.Hk, self.max_c)
+        self.P = partition or api.default_partition(self.S, self.Hk, self.max_c)
         self.workspace = api.alloc_workspace(self.S, self.H, self.Hk, self.d, self.max_c, self.P, device)
 
     def _lengths(self):
@@ -136,9 +136,9 @@ class SharedPrefixWorkload(Workload):
 
     REQUESTS, WIDTH, PROMPT, TAIL_MAX = 32, 4, 1024, 256
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0):
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0):
         self.rnd = torch.Generator().manual_seed(4 + seed_offset)
-        super().__init__(name, device, seed_offset, growth_steps + 64)
+        super().__init__(name, device, seed_offset, growth_steps + 64, partition)
 
     def _lengths(self):
         tails = torch.randint(0, self.TAIL_MAX + 1, (self.REQUESTS * self.WIDTH,), generator=self.rnd)
@@ -186,9 +186,9 @@ class SharedPrefixWorkload(Workload):
         return len(used) * self.Hk * self.B * self.d * 2 * self.es
 
 
-def make_workload(name, device, seed_offset=0, growth_steps=0):
+def make_workload(name, device, seed_offset=0, growth_steps=0, partition=0):
     cls = SharedPrefixWorkload if name == "shared_prefix_bf16" else Workload
-    return cls(name, device, seed_offset, growth_steps)
+    return cls(name, device, seed_offset, growth_steps, partition)
 
 
 def load_peaks():
@@ -289,7 +289,8 @@ def run_pa(args, rank, world, local_rank):
     K, Wm = args.steps, args.warmup
     e2e_steps = min(K, args.e2e_steps)
     n_traj = 32 if args.workload == "shared_prefix_bf16" else 1
-    wl = make_workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + n_traj + 2)
+    wl = make_workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + n_traj + 2,
+                       partition=args.partition)
     S, H, Hk, d = wl.S, wl.H, wl.Hk, wl.d
     gen = torch.Generator(device=dev).manual_seed(99 + rank)
     q = torch.randn((S, H, d), generator=gen, device=dev).to(wl.dtype)
@@ -355,48 +356,26 @@ def run_pa(args, rank, world, local_rank):
     lens = traj[0]["lens"].cpu()
     launches_total = sum(launches[i % n_traj] for i in range(K))
 
-    # ---- end to end through the API, from pinned host memory ----
-    pin = lambda t: t.cpu().pin_memory()
-    h_q, h_key, h_val = pin(q), pin(key), pin(val)
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_slots = torch.empty(S, dtype=torch.int64).pin_memory()
-    h_pairs = torch.empty((S, 2), dtype=torch.int32).pin_memory()
-    h_tables = torch.empty((S, wl.max_blocks), dtype=torch.int32).pin_memory()
-    h_lens = torch.empty(S, dtype=torch.int32).pin_memory()
-    d_q, d_key, d_val = torch.empty_like(q), torch.empty_like(key), torch.empty_like(val)
-    d_slots2 = torch.empty(S, dtype=torch.int64, device=dev)
-    d_pairs2 = torch.empty((S, 2), dtype=torch.int32, device=dev)
-    d_tables2 = torch.empty((S, wl.max_blocks), dtype=torch.int32, device=dev)
-    d_lens2 = torch.empty(S, dtype=torch.int32, device=dev)
+    # ---- end to end through the API: one captured step per iteration, from pinned host memory ----
+    step = api.DecodeStep(wl.k_cache, wl.v_cache, S, H, wl.max_blocks, wl.max_c, max_pairs=S, out_dtype=wl.dtype,
+                          partition_size=wl.P)
+    step.h_query.copy_(q.cpu())
+    step.h_key.copy_(key.cpu())
+    step.h_value.copy_(val.cpu())
+    es, B = wl.es, wl.B
     e2e_bytes = 0
-    h2d = d2h = 0
 
     def e2e_step():
-        nonlocal e2e_bytes, h2d, d2h
-        sl, pr, tb, ln = wl.host_step(h_slots, h_pairs, h_tables, h_lens)
-        npairs = pr.shape[0]
-        d_q.copy_(h_q, non_blocking=True)
-        d_key.copy_(h_key, non_blocking=True)
-        d_val.copy_(h_val, non_blocking=True)
-        d_slots2.copy_(sl, non_blocking=True)
-        d_tables2.copy_(tb, non_blocking=True)
-        d_lens2.copy_(ln, non_blocking=True)
-        moved = [h_q, h_key, h_val, sl, tb, ln]
-        if npairs:
-            d_pairs2[:npairs].copy_(pr, non_blocking=True)
-            moved.append(pr)
-            api.pa_copy_blocks(wl.k_cache, wl.v_cache, d_pairs2[:npairs])
-        api.pa_cache_write(wl.k_cache, wl.v_cache, d_key, d_val, d_slots2)
-        api.pa_decode(d_q, wl.k_cache, wl.v_cache, d_tables2, d_lens2, max_context_len=wl.max_c, out=out,
-                      partition_size=wl.P, workspace=wl.workspace)
-        h_out.copy_(out, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        e2e_bytes += wl.step_bytes(ln.tolist(), npairs)[1]
-        h2d += sum(t.numel() * t.element_size() for t in moved)
-        d2h += h_out.numel() * h_out.element_size()
+        nonlocal e2e_bytes
+        _, pr, _, ln = wl.host_step(step.h_slots, None, step.h_tables, step.h_lens)
+        step.set_pairs(pr)
+        step.run()
+        c_sum, nb_sum = int(ln.sum()), int(((ln + (B - 1)) // B).sum())
+        e2e_bytes += (c_sum * Hk * d * 2 * es + S * H * d * es * 2 + 4 * nb_sum + 4 * S
+                      + 2 * (S * Hk * d * es * 2) + 8 * S + pr.shape[0] * 2 * (Hk * B * d * es) * 2)
 
     e2e_step()  # warm-up (also grows every sequence by one token)
-    e2e_bytes = h2d = d2h = 0
+    e2e_bytes = 0
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -408,6 +387,7 @@ def run_pa(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clocks.mark(t_wall0, time.time())
+    h2d, d2h = step.h2d_bytes * e2e_steps, step.d2h_bytes * e2e_steps
     e2e_ms = e0.elapsed_time(e1)
     clock_info = clocks.finish()
 
@@ -473,7 +453,8 @@ def run_pa(args, rank, world, local_rank):
             "d2h_bytes_per_step": d2h // max(e2e_steps, 1),
             "steps": e2e_steps,
             "ms_per_step": round(e2e_ms / e2e_steps, 5),
-            "note": "host block manager + H2D of the step's inputs + kernels + D2H of o, synchronised each step",
+            "note": "per step: host block manager, then one replay of the captured step (H2D of the step's "
+                    "inputs from pinned memory, copy_blocks, cache_write, decode, D2H of o), synchronised",
         },
         "gpu_launches": launches_total,
     }
@@ -531,6 +512,140 @@ def cpu_baseline(wl, lens, q, target_s=12.0):
     return {"value": round(byt / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{passes} pass(es) over {len(sample)} of {wl.S} sequences ({sum(c)} tokens x {H} heads), "
                       f"decode only, fp64 C++ oracle with {cores} threads, {dt:.1f} s"}
+
+
+def run_swap(args, rank, world, local_rank):
+    """Preemption by swapping: K steps of (swap 512 blocks out to pinned host memory, swap them
+    back in), gqa8k-shaped blocks (8 kv heads x 16 tokens x 128 dims, bf16: 64 KiB per block for K
+    and V).  The roofline is the host link, measured in the same run as pinned copies of the same
+    bytes in each direction."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    n_dev, n_host, n_swap, Hk, B, d, dt = 4096, 1024, 512, 8, 16, 128, torch.bfloat16
+    gen = torch.Generator(device=dev).manual_seed(11 + rank)
+    dk = torch.randn((n_dev, Hk, B, d), generator=gen, device=dev).to(dt)
+    dv = torch.randn((n_dev, Hk, B, d), generator=gen, device=dev).to(dt)
+    hk = torch.empty((n_host, Hk, B, d), dtype=dt).pin_memory()
+    hv = torch.empty((n_host, Hk, B, d), dtype=dt).pin_memory()
+    g = torch.Generator().manual_seed(12)
+    src = torch.randperm(n_dev, generator=g)[:n_swap]
+    out_pairs = torch.stack([src, torch.randperm(n_host, generator=g)[:n_swap]], 1).to(torch.int32).to(dev)
+    back = torch.randperm(n_dev, generator=g)[:n_swap]
+    in_pairs = torch.stack([out_pairs[:, 1].cpu(), back], 1).to(torch.int32).to(dev)
+    blk_bytes = Hk * B * d * 2
+    moved = 2 * n_swap * blk_bytes * 2          # K and V, out and in
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def step():
+        api.pa_swap_blocks(hk, hv, dk, dv, out_pairs)
+        api.pa_swap_blocks(dk, dv, hk, hv, in_pairs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    t0 = time.time()
+    ev[0].record()
+    for _ in range(args.steps):
+        step()
+    ev[1].record()
+    torch.cuda.synchronize()
+    clocks.mark(t0, time.time())
+    ms = ev[0].elapsed_time(ev[1])
+    # host-link reference: plain pinned copies of the same number of bytes, each direction
+    a = torch.empty(n_swap * blk_bytes * 2, dtype=torch.uint8, device=dev)
+    h = torch.empty(a.numel(), dtype=torch.uint8).pin_memory()
+    for _ in range(3):
+        h.copy_(a, non_blocking=True)
+        a.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    ev[2].record()
+    for _ in range(args.steps):
+        h.copy_(a, non_blocking=True)
+        a.copy_(h, non_blocking=True)
+    ev[3].record()
+    torch.cuda.synchronize()
+    ref_ms = ev[2].elapsed_time(ev[3])
+    clock_info = clocks.finish()
+    ms, ref_ms = reduce_max([ms, ref_ms], world, dev)
+    if rank != 0:
+        return None
+    value = aggregate_value(moved, args.steps, world, ms)
+    peak = aggregate_value(moved, args.steps, world, ref_ms) / world
+    return {"metric": "block swap GB/s (device <-> pinned host, out and back in)", "value": round(value, 2),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"swap {n_swap} blocks of 8x16x128 bf16 out to pinned host memory and back",
+                       "step_bytes": moved},
+            "roofline": {"bound": "host link", "achieved": round(value / world, 2), "peak": round(peak, 2),
+                         "peak_kind": "pinned torch copies of the same bytes, same run", "unit": "GB/s",
+                         "frac": round(value / world / peak, 4), "traffic": None},
+            "clocks": clock_info, "gpu_launches": 2 * args.steps}
+
+
+def run_prefill(args, rank, world, local_rank):
+    """Mixed batch through pa_prefill: 16 prompt chunks of 512 tokens at the end of contexts
+    U[1024, 4096] plus 64 decode tokens with lognormal contexts (median 1024), GQA 32/8, d 128,
+    B 16, bf16.  FLOPs = 4 d (p + 1) per (query token, head) at position p (q.k and p.v of the
+    causal prefix); compared with the measured dense bf16 tensor peak."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    H, Hk, d, B, dt = 32, 8, 128, 16, torch.bfloat16
+    g = W.generator(21 + rank)
+    ctx_p = W.lens_uniform(g, 16, 1024, 4096).tolist()
+    ctx_d = W.lens_lognormal(g, 64, 1024.0, 1.0, 16, 8192).tolist()
+    ctx = ctx_p + ctx_d
+    nq = [512] * 16 + [1] * 64
+    case = W.paged_case("prefill", ctx, H, Hk, d, B, dt, 21 + rank, sentinel="none", device=dev)
+    q_start = torch.tensor([0] + list(torch.tensor(nq).cumsum(0)), dtype=torch.int32, device=dev)
+    q = torch.randn((int(q_start[-1]), H, d), generator=torch.Generator(device=dev).manual_seed(5), device=dev).to(dt)
+    max_c, max_q = max(ctx), max(nq)
+    ws = torch.empty(api._native.load().pa_prefill_workspace_size(len(ctx), H, Hk, max_q), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty_like(q)
+    flops = sum(4 * d * H * sum(c - n + i + 1 for i in range(n)) for c, n in zip(ctx, nq))
+    kv_bytes = sum(ctx) * Hk * d * 2 * 2
+
+    def step():
+        api.pa_prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                       max_context_len=max_c, max_q_len=max_q, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert api.workspace_error(ws) == 0
+    clocks = ClockSampler(local_rank)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks.mark(t0, time.time())
+    ms = e0.elapsed_time(e1)
+    clock_info = clocks.finish()
+    (ms,) = reduce_max([ms], world, dev)
+    if rank != 0:
+        return None
+    tflops = world * flops * args.steps / (ms * 1e-3) / 1e12
+    try:
+        peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+        kind = "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    return {"metric": "paged prefill + decode attention TFLOP/s (mixed batch)", "value": round(tflops, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "16 prompt chunks of 512 tokens (contexts U[1024,4096]) + 64 decode tokens "
+                                   "(lognormal contexts), 32/8 heads, d 128, B 16",
+                       "flops_per_step": flops, "unique_kv_bytes": kv_bytes},
+            "kv_gbs_unique": round(world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, 2),
+            "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak, "peak_kind": kind,
+                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4), "traffic": None},
+            "clocks": clock_info, "gpu_launches": 2 * args.steps}
 
 
 def run_reference(args, rank, world):
@@ -606,8 +721,9 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
-    ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS) + ["swap_bf16", "prefill_mixed_bf16"])
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--partition", type=int, default=0, help="decode partition size in tokens (0 = library default)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -625,8 +741,14 @@ def main():
             torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     try:
-        if args.impl == "reference":
+        if args.impl == "reference" and args.workload in ("swap_bf16", "prefill_mixed_bf16"):
+            line = {"impl": "reference", "unavailable": "the oracle arm times the decode workloads only"} if rank == 0 else None
+        elif args.impl == "reference":
             line = run_reference(args, rank, world)
+        elif args.workload == "swap_bf16":
+            line = run_swap(args, rank, world, local_rank)
+        elif args.workload == "prefill_mixed_bf16":
+            line = run_prefill(args, rank, world, local_rank)
         else:
             from paged_kv_cache_329_b200 import build
 

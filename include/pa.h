@@ -186,6 +186,105 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
                          int B, int n_blocks, pa_dtype dtype, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Paged attention for several query tokens per sequence: chunked prefill, and batches that mix
+ * prefill chunks with decode tokens ("vllm" 2.1 Prefill: the prompt's tokens are processed
+ * together; "Paged Attention&Orca Paper笔记与解读", selective batching: tokens of requests in
+ * different phases are batched and only attention separates them).
+ *
+ * Sequence s has n_s = q_start[s+1] - q_start[s] query tokens (rows q_start[s] .. q_start[s+1]-1 of
+ * query), which are the LAST n_s of its c_s = context_lens[s] tokens and are already in the cache
+ * (pa_cache_write first).  The token at position p = c_s - n_s + i attends to positions 0 .. p:
+ *     out[row][h] = softmax(scale * q K[0..p]^T) V[0..p]      (kv head h / (H/Hk)),
+ * the decode definition with the context cut at the token's own position; n_s = 1 is exactly
+ * pa_decode.  Needs n_s <= c_s, n_s <= max_q_len, c_s <= max_context_len; values outside
+ * are cut to those bounds and set bit 2 of the workspace error word.
+ *
+ *   out           device [T][H][d] of out_dtype, T = q_start[S]
+ *   query         device [T][H][d] of kv_dtype (fp16 or bf16 only)
+ *   q_start       device [S+1] int32, non-decreasing, q_start[0] = 0
+ *   k_cache, v_cache, block_tables, context_lens, B, n_blocks, max_blocks_per_seq: as pa_decode
+ *   max_q_len     host bound on every n_s
+ *   workspace     device scratch of pa_prefill_workspace_size(...) bytes, 256-byte aligned
+ */
+size_t pa_prefill_workspace_size(int S, int H, int Hk, int max_q_len);
+
+pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
+                     const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int S, int H, int Hk, int d, int B, int n_blocks,
+                     int max_blocks_per_seq, int max_context_len, int max_q_len, float scale,
+                     pa_dtype kv_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Block swap for preemption by swapping ("PagedAttention原理", "抢占与恢复", swap: a preempted
+ * sequence's blocks move to CPU memory and are moved back before it runs again; the CPU pool is at
+ * most as large as the GPU pool).  For each pair p: block pairs[p][1] of the destination pool
+ * becomes a bit copy of block pairs[p][0] of the source pool, for K and for V.  Both pools have the
+ * [n][Hk][B][d] layout of the caches; one is normally the device cache and the other pinned host
+ * memory (cudaHostAlloc / cudaHostRegister), which the kernel reads or writes over the host link.
+ * Destination blocks must be distinct.  Out-of-range ids are skipped.
+ *
+ *   dst_k, dst_v  [n_dst_blocks][Hk][B][d], device or pinned host
+ *   src_k, src_v  [n_src_blocks][Hk][B][d], device or pinned host
+ *   pairs         [P][2] int32 (src, dst), device or pinned host
+ */
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, int n_dst_blocks, const void* src_k, const void* src_v,
+                         int n_src_blocks, const int32_t* pairs, int P, int Hk, int d, int B, pa_dtype dtype,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * A whole decode step as one replayable CUDA graph.
+ *
+ * One step of serving, in stream order: copy the step's inputs from pinned host buffers to the
+ * device, pa_copy_blocks on the step's copy-on-write pairs, pa_cache_write of one new token per
+ * sequence, pa_decode, and copy the output back to the host.  pa_step_create captures this once
+ * into a CUDA graph over the fixed buffers named in the descriptor; pa_step_run replays it, so a
+ * step costs one graph launch instead of a dozen API calls (the copy-on-write count, which varies
+ * from step to step, travels in pinned memory with the other inputs).  The caller refills the host
+ * buffers (e.g. with pa_seq_reserve_slots_batch and pa_build_block_tables) before each run.
+ */
+typedef struct {
+  /* pinned host buffers (cudaHostAlloc / cudaHostRegister memory), read or written by each run */
+  const void* h_query;          /* [S][H][d] kv_dtype */
+  const void* h_key;            /* [S][Hk][d] kv_dtype: the new token of each sequence */
+  const void* h_value;          /* [S][Hk][d] kv_dtype */
+  const int64_t* h_slots;       /* [S] slot of each new token (< 0: no token) */
+  const int32_t* h_pairs;       /* [max_pairs][2] copy-on-write (src, dst) pairs */
+  const int32_t* h_n_pairs;     /* one int: pairs used this step, 0 .. max_pairs */
+  const int32_t* h_tables;      /* [S][max_blocks_per_seq] */
+  const int32_t* h_lens;        /* [S] context lengths including the new token */
+  void* h_out;                  /* [S][H][d] out_dtype, written by each run */
+  /* device buffers (the same sizes), plus the caches and a decode workspace */
+  void* d_query;
+  void* d_key;
+  void* d_value;
+  int64_t* d_slots;
+  int32_t* d_pairs;             /* [max_pairs][2] followed by one int (the count): 8*max_pairs+16 bytes */
+  int32_t* d_tables;
+  int32_t* d_lens;
+  void* d_out;
+  void* k_cache;
+  void* v_cache;
+  void* workspace;
+  size_t workspace_bytes;
+  /* sizes */
+  int S, H, Hk, d, B, n_blocks, max_blocks_per_seq, max_context_len, max_pairs, partition_size;
+  float scale;
+  pa_dtype kv_dtype, out_dtype;
+} pa_step_desc;
+
+typedef struct pa_step pa_step;
+
+/* Validates the descriptor, captures the step into a graph (on a private stream of the current
+ * device) and instantiates it.  The capture itself runs nothing.  Every host buffer must be pinned.
+ * NULL on failure (pa_last_error() says why). */
+pa_step* pa_step_create(const pa_step_desc* desc);
+
+/* Launches the captured step on `stream` and waits for it (the output is in h_out on return). */
+pa_status pa_step_run(pa_step* step, void* stream);
+
+void pa_step_destroy(pa_step* step);
+
+/* ---------------------------------------------------------------------------------------------
  * Host block manager ("从虚拟内存的启发", "解决共享prompt", "解决COW", "COW 区别").  Pure CPU; a handle
  * must not be used by two threads at once.  Policies (the pages leave them open):
  *   - free blocks form a LIFO stack that starts as [n_blocks-1, ..., 1, 0]: the first allocation

@@ -14,6 +14,9 @@ Pages followed (title, section, equation):
     partials(), combine()
   * "vllm" (cnblogs), 2.2 Decode: the new token's K,V are stored in the cache -> cache_write()
   * "PagedAttention原理", "解决COW", step 2 (copy the shared block)        -> copy_blocks()
+  * "PagedAttention原理", "抢占与恢复", swap (blocks to CPU memory and back)  -> swap_blocks()
+  * Orca notes (selective batching) and "vllm" 2.1 Prefill: several causal query tokens per
+    sequence, decode being one                                                -> prefill()
 """
 from __future__ import annotations
 
@@ -56,6 +59,10 @@ def _declare(lib):
     lib.oracle_cache_write.restype = I
     lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I]
     lib.oracle_copy_blocks.restype = I
+    lib.oracle_prefill.argtypes = [P, P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, D, I]
+    lib.oracle_prefill.restype = I
+    lib.oracle_swap_blocks.argtypes = [P, P, I, P, P, I, P, I, I, I, I, I]
+    lib.oracle_swap_blocks.restype = I
     lib.oracle_hardware_threads.argtypes = []
     lib.oracle_hardware_threads.restype = I
     lib.oracle_elem_to_double.argtypes = [P, I, L]
@@ -213,3 +220,37 @@ def copy_blocks(k_cache, v_cache, pairs):
     if rc != 0:
         raise ValueError("oracle_copy_blocks: block id out of range")
     return kc, vc
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, pairs):
+    """Whole-block copies from a source pool into copies of a destination pool; returns (dst_k', dst_v')."""
+    dk, dv = _cpu(dst_k).clone(), _cpu(dst_v).clone()
+    sk, sv = _cpu(src_k), _cpu(src_v)
+    pr = _cpu(pairs.to(torch.int32).reshape(-1, 2))
+    n_dst, Hk, B, d = dk.shape
+    if sk.shape[1:] != dk.shape[1:] or sk.dtype != dk.dtype:
+        raise ValueError("pools must share the block layout and type")
+    rc = _L().oracle_swap_blocks(dk.data_ptr(), dv.data_ptr(), n_dst, sk.data_ptr(), sv.data_ptr(), sk.shape[0],
+                                 pr.data_ptr(), pr.shape[0], Hk, d, B, _code(dk))
+    if rc != 0:
+        raise ValueError("oracle_swap_blocks: block id out of range")
+    return dk, dv
+
+
+def prefill(q, q_start, k_cache, v_cache, block_tables, context_lens, scale=None, n_threads=1):
+    """Causal attention of each sequence's last n_s tokens over its paged context; [T, H, d] fp64."""
+    q, k_cache, v_cache = _cpu(q), _cpu(k_cache), _cpu(v_cache)
+    qs = _cpu(q_start.to(torch.int32))
+    bt, cl = _cpu(block_tables.to(torch.int32)), _cpu(context_lens.to(torch.int32))
+    T, H, d = q.shape
+    n_blocks, Hk, B, d2 = k_cache.shape
+    S = cl.numel()
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    out = torch.empty((T, H, d), dtype=torch.float64)
+    rc = _L().oracle_prefill(out.data_ptr(), q.data_ptr(), _code(q), qs.data_ptr(), k_cache.data_ptr(),
+                             v_cache.data_ptr(), _code(k_cache), bt.data_ptr(), cl.data_ptr(), S, H, Hk, d, B,
+                             n_blocks, bt.shape[1], float(scale), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill failed ({rc})")
+    return out

@@ -334,4 +334,74 @@ int oracle_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int P
   return 0;
 }
 
+// Chunked prefill and mixed batches ("Paged Attention&Orca Paper笔记与解读", selective batching:
+// prefill and decode tokens of different requests are batched, and only attention needs to know
+// each token's request and phase; "vllm" 2.1 Prefill: the prompt's tokens are processed together).
+// Sequence s has n_s = q_start[s+1] - q_start[s] query tokens, the last n_s of its c_s context
+// tokens (already in the cache); the token at position p = c_s - n_s + i attends to positions
+// 0..p (causal), i.e. o = softmax(scale * q K[0..p]^T) V[0..p] -- the decode definition applied
+// to each query token with the context cut at its own position.  Decode is n_s = 1.
+// query: [T][H][d]; out: [T][H][d] doubles.  Returns -1 on a bad table entry or n_s > c_s.
+int oracle_prefill(double* out, const void* q, int q_dtype, const int32_t* q_start, const void* k_cache,
+                   const void* v_cache, int kv_dtype, const int32_t* block_tables, const int32_t* context_lens,
+                   int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq, double scale,
+                   int n_threads) {
+  if (S < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || d <= 0 || B <= 0) return -2;
+  const int g = H / Hk;
+  const int T = S > 0 ? q_start[S] : 0;
+  std::atomic<int> bad{0};
+  parallel_for(static_cast<long>(T) * H, n_threads, [&](long u) {
+    const int row = static_cast<int>(u / H), h = static_cast<int>(u % H), kh = h / g;
+    int s = 0;
+    while (s + 1 <= S && q_start[s + 1] <= row) ++s;  // the sequence this query token belongs to
+    const int n = q_start[s + 1] - q_start[s], c = context_lens[s];
+    double* o = out + (static_cast<size_t>(row) * H + h) * d;
+    for (int i = 0; i < d; ++i) o[i] = 0.0;
+    if (n > c) {
+      bad = 1;
+      return;
+    }
+    const int pos = c - n + (row - q_start[s]);  // this token's position; it sees 0..pos
+    std::vector<double> qv(d), x(pos + 1);
+    for (int i = 0; i < d; ++i) qv[i] = load_elem(q, q_dtype, (static_cast<size_t>(row) * H + h) * d + i);
+    double mx = -INFINITY;
+    std::vector<size_t> rows(pos + 1);
+    for (int t = 0; t <= pos; ++t) {
+      if (!token_row(block_tables, max_blocks_per_seq, n_blocks, s, t, Hk, kh, B, &rows[t])) {
+        bad = 1;
+        return;
+      }
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += qv[i] * load_elem(k_cache, kv_dtype, rows[t] * d + i);
+      x[t] = scale * acc;
+      if (x[t] > mx) mx = x[t];
+    }
+    double z = 0.0;
+    for (int t = 0; t <= pos; ++t) {
+      x[t] = std::exp(x[t] - mx);
+      z += x[t];
+    }
+    for (int t = 0; t <= pos; ++t)
+      for (int i = 0; i < d; ++i) o[i] += x[t] * load_elem(v_cache, kv_dtype, rows[t] * d + i);
+    for (int i = 0; i < d; ++i) o[i] /= z;
+  });
+  return bad ? -1 : 0;
+}
+
+// Preemption by swapping ("PagedAttention原理", "抢占与恢复", swap: a preempted sequence's blocks move
+// to CPU memory and come back before it runs again): for each (src, dst) pair, block dst of the
+// destination pool becomes a copy of block src of the source pool, for K and V.  The two pools
+// have the same [n][Hk][B][d] layout and may differ in size.  Returns -1 on an out-of-range id.
+int oracle_swap_blocks(void* dst_k, void* dst_v, int n_dst, const void* src_k, const void* src_v, int n_src,
+                       const int32_t* pairs, int P, int Hk, int d, int B, int dtype) {
+  const size_t bytes = static_cast<size_t>(Hk) * B * d * elem_bytes(dtype);
+  for (int p = 0; p < P; ++p) {
+    const int32_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+    if (src < 0 || src >= n_src || dst < 0 || dst >= n_dst) return -1;
+    std::memcpy(static_cast<char*>(dst_k) + dst * bytes, static_cast<const char*>(src_k) + src * bytes, bytes);
+    std::memcpy(static_cast<char*>(dst_v) + dst * bytes, static_cast<const char*>(src_v) + src * bytes, bytes);
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -7,6 +7,7 @@ computes on the CPU.
 """
 from .api import (  # noqa: F401
     BlockManager,
+    DecodeStep,
     NoFreeBlock,
     PAError,
     alloc_workspace,
@@ -16,6 +17,8 @@ from .api import (  # noqa: F401
     pa_combine,
     pa_copy_blocks,
     pa_decode,
+    pa_prefill,
+    pa_swap_blocks,
     version,
     workspace_error,
 )

@@ -19,6 +19,19 @@ I32P = ctypes.POINTER(ctypes.c_int32)
 I64P = ctypes.POINTER(ctypes.c_int64)
 IP = ctypes.POINTER(ctypes.c_int)
 
+class StepDesc(ctypes.Structure):
+    """pa_step_desc of include/pa.h, field for field."""
+    _fields_ = [
+        ("h_query", P), ("h_key", P), ("h_value", P), ("h_slots", P), ("h_pairs", P), ("h_n_pairs", P),
+        ("h_tables", P), ("h_lens", P), ("h_out", P),
+        ("d_query", P), ("d_key", P), ("d_value", P), ("d_slots", P), ("d_pairs", P), ("d_tables", P),
+        ("d_lens", P), ("d_out", P), ("k_cache", P), ("v_cache", P), ("workspace", P), ("workspace_bytes", SZ),
+        ("S", I), ("H", I), ("Hk", I), ("d", I), ("B", I), ("n_blocks", I), ("max_blocks_per_seq", I),
+        ("max_context_len", I), ("max_pairs", I), ("partition_size", I),
+        ("scale", F), ("kv_dtype", I), ("out_dtype", I),
+    ]
+
+
 # name -> (restype, argtypes); mirrors include/pa.h
 SIGNATURES = {
     "pa_last_error": (ctypes.c_char_p, []),
@@ -27,10 +40,16 @@ SIGNATURES = {
     "pa_decode": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
     "pa_decode_noalloc": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P]),
     "pa_decode_default_partition": (I, [I, I, I]),
+    "pa_prefill_workspace_size": (SZ, [I, I, I, I]),
+    "pa_prefill": (I, [P, I, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, SZ, P]),
     "pa_workspace_error": (I, [P, IP, P]),
     "pa_combine": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),
     "pa_cache_write": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
     "pa_copy_blocks": (I, [P, P, P, I, I, I, I, I, I, P]),
+    "pa_swap_blocks": (I, [P, P, I, P, P, I, P, I, I, I, I, I, P]),
+    "pa_step_create": (P, [ctypes.POINTER(StepDesc)]),
+    "pa_step_run": (I, [P, P]),
+    "pa_step_destroy": (None, [P]),
     "pa_alloc_create": (P, [I, I]),
     "pa_alloc_destroy": (None, [P]),
     "pa_alloc_block": (I, [P, I32P]),

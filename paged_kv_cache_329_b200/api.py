@@ -93,6 +93,30 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, *, max_context_le
     return out
 
 
+def pa_prefill(q, q_start, k_cache, v_cache, block_tables, context_lens, *, max_context_len, max_q_len,
+               scale=None, out=None, out_dtype=None, workspace=None, stream=None):
+    """Causal paged attention for several query tokens per sequence (prefill chunks and decode tokens
+    in one batch); returns out [T, H, d].  See pa_prefill in include/pa.h."""
+    _cuda(q, q_start, k_cache, v_cache, block_tables, context_lens)
+    T, H, d = q.shape
+    n_blocks, Hk, B, d2 = k_cache.shape
+    S = context_lens.numel()
+    if d2 != d or q.dtype != k_cache.dtype or q_start.dtype != torch.int32 or q_start.numel() != S + 1:
+        raise ValueError("shape/dtype mismatch")
+    if out is None:
+        out = torch.empty((T, H, d), dtype=out_dtype or q.dtype, device=q.device)
+    if workspace is None:
+        n = _native.load().pa_prefill_workspace_size(S, H, Hk, int(max_q_len))
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(_native.load().pa_prefill(
+        _ptr(out), DTYPE[out.dtype], _ptr(q), _ptr(q_start), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), S, H, Hk, d, B, n_blocks, block_tables.shape[1], int(max_context_len), int(max_q_len),
+        float(scale), DTYPE[q.dtype], _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def workspace_error(workspace, stream=None) -> int:
     flags = ctypes.c_int(0)
     _check(_native.load().pa_workspace_error(_ptr(workspace), ctypes.byref(flags), _stream(stream)))
@@ -132,6 +156,91 @@ def pa_copy_blocks(k_cache, v_cache, pairs, stream=None):
     _check(_native.load().pa_copy_blocks(
         _ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.numel() // 2, Hk, d, B, n_blocks,
         DTYPE[k_cache.dtype], _stream(stream)))
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, stream=None):
+    """Whole-block copies between the device cache and a pinned host pool (either direction)."""
+    for t in (dst_k, dst_v, src_k, src_v, pairs):
+        if not t.is_contiguous() or not (t.is_cuda or t.is_pinned()):
+            raise ValueError("pools and pairs must be contiguous CUDA or pinned host tensors")
+    n_dst, Hk, B, d = dst_k.shape
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype or pairs.dtype != torch.int32:
+        raise ValueError("pools must share the block layout and type; pairs int32 [P, 2]")
+    _check(_native.load().pa_swap_blocks(
+        _ptr(dst_k), _ptr(dst_v), n_dst, _ptr(src_k), _ptr(src_v), src_k.shape[0], _ptr(pairs),
+        pairs.numel() // 2, Hk, d, B, DTYPE[dst_k.dtype], _stream(stream)))
+
+
+# ---- a decode step as one CUDA graph -------------------------------------------------------------
+
+class DecodeStep:
+    """pa_step_*: the step's H2D copies, COW copy, cache write, decode and D2H of o, captured once.
+
+    Fill the pinned host tensors (h_query, h_key, h_value, h_slots, h_pairs, h_n_pairs, h_tables,
+    h_lens) before each run(); the output is in h_out afterwards.
+    """
+
+    def __init__(self, k_cache, v_cache, S, H, max_blocks_per_seq, max_context_len, *, max_pairs=None,
+                 out_dtype=None, scale=None, partition_size=0):
+        _cuda(k_cache, v_cache)
+        n_blocks, Hk, B, d = k_cache.shape
+        dt, dev = k_cache.dtype, k_cache.device
+        out_dtype = out_dtype or dt
+        max_pairs = S if max_pairs is None else max_pairs
+        pin = lambda shape, t: torch.empty(shape, dtype=t).pin_memory()
+        self.h_query, self.h_key, self.h_value = pin((S, H, d), dt), pin((S, Hk, d), dt), pin((S, Hk, d), dt)
+        self.h_slots = pin((S,), torch.int64)
+        self.h_pairs = pin((max(max_pairs, 1), 2), torch.int32)
+        self.h_n_pairs = pin((1,), torch.int32)
+        self.h_tables = pin((S, max_blocks_per_seq), torch.int32)
+        self.h_lens = pin((S,), torch.int32)
+        self.h_out = pin((S, H, d), out_dtype)
+        self.h_n_pairs.zero_()
+        self.h_slots.fill_(-1)
+        self.h_lens.zero_()
+        dz = lambda shape, t: torch.zeros(shape, dtype=t, device=dev)
+        self.d_query, self.d_key, self.d_value = dz((S, H, d), dt), dz((S, Hk, d), dt), dz((S, Hk, d), dt)
+        self.d_slots = dz((S,), torch.int64)
+        self.d_pairs = dz((2 * max(max_pairs, 1) + 4,), torch.int32)
+        self.d_tables = dz((S, max_blocks_per_seq), torch.int32)
+        self.d_lens = dz((S,), torch.int32)
+        self.d_out = dz((S, H, d), out_dtype)
+        self.workspace = alloc_workspace(S, H, Hk, d, max_context_len, partition_size, dev)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        vp = lambda t: t.data_ptr()
+        desc = _native.StepDesc(
+            vp(self.h_query), vp(self.h_key), vp(self.h_value), vp(self.h_slots), vp(self.h_pairs),
+            vp(self.h_n_pairs), vp(self.h_tables), vp(self.h_lens), vp(self.h_out),
+            vp(self.d_query), vp(self.d_key), vp(self.d_value), vp(self.d_slots), vp(self.d_pairs),
+            vp(self.d_tables), vp(self.d_lens), vp(self.d_out), vp(k_cache), vp(v_cache), vp(self.workspace),
+            self.workspace.numel(), S, H, Hk, d, B, n_blocks, max_blocks_per_seq, max_context_len, max_pairs,
+            partition_size, float(1.0 / math.sqrt(d) if scale is None else scale), DTYPE[dt], DTYPE[out_dtype])
+        self._lib = _native.load()
+        self._h = self._lib.pa_step_create(ctypes.byref(desc))
+        if not self._h:
+            raise PAError(PA_ERR_INVALID_ARG, self._lib.pa_last_error().decode())
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
+                             (self.h_query, self.h_key, self.h_value, self.h_slots, self.h_pairs, self.h_n_pairs,
+                              self.h_tables, self.h_lens))
+        self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
+
+    def set_pairs(self, pairs):
+        n = int(pairs.shape[0]) if pairs is not None else 0
+        if n > self.h_pairs.shape[0]:
+            raise ValueError("more copy-on-write pairs than max_pairs")
+        if n:
+            self.h_pairs[:n].copy_(pairs)
+        self.h_n_pairs[0] = n
+
+    def run(self, stream=None):
+        _check(self._lib.pa_step_run(self._h, _stream(stream)))
+        return self.h_out
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            self._lib.pa_step_destroy(h)
+            self._h = None
 
 
 # ---- host block manager -------------------------------------------------------------------------

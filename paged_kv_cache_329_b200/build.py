@@ -23,7 +23,7 @@ OBJ_DIR = os.path.join(ROOT, "_build", "libpa")
 LIB = os.path.join(HERE, "libpa.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["pa_error.cpp", "pa_alloc.cpp", "pa_cache.cu", "pa_decode.cu"]
+SOURCES = ["pa_error.cpp", "pa_alloc.cpp", "pa_cache.cu", "pa_decode.cu", "pa_prefill.cu", "pa_step.cu"]
 
 
 def _nvcc() -> str:

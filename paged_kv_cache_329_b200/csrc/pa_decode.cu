@@ -33,6 +33,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -101,63 +102,68 @@ WsLayout ws_layout(int S, int H, int Hk, int d, int max_parts) {
 }
 
 // ---- plan: list the work units -----------------------------------------------------------------
-// Unit order: every whole partition (parts 0 .. n_parts-2 of each sequence), ordered by
-// (sequence, part, kv head), then every sequence's last partition, ordered by (sequence, kv head).
-// n_parts(s) = max(1, ceil(c / P)); c = 0 still gets one unit, which writes zeros.
+// Units are (sequence, kv head, partition); n_parts(s) = max(1, ceil(c / P)) and c = 0 still gets
+// one unit, which writes zeros.  Units are listed longest first (by 64-token tiles, in at most
+// kBuckets groups): every whole partition, then the last partitions from longest to shortest, so
+// the persistent grid ends on short units.  Positions inside a group come from atomic cursors;
+// the order of units does not change any result (each unit's arithmetic is independent of it, and
+// partitions are merged in index order).
+constexpr int kBuckets = 64;
+
+__device__ __forceinline__ int tile_bucket(int ntok, int P) {
+  const int tiles = (ntok + kTileTokens - 1) / kTileTokens;  // 0 .. P/64
+  const int max_tiles = P / kTileTokens;
+  const int nb = max_tiles < kBuckets ? max_tiles : kBuckets;
+  return tiles <= 1 ? 0 : ((tiles - 1) * nb) / max_tiles;    // 0 .. nb-1, monotone in ntok
+}
+
+constexpr int kPlanCache = 4096;  // lengths kept in shared memory between the two passes
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ lens, int S, int Hk, int P,
                                                             int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
-  __shared__ int warp_tot[kPlanThreads / 32];
-  __shared__ int chunk_total;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  int base = 0;  // whole partitions listed so far (in units of (s, part), before the Hk factor)
-  for (int s0 = 0; s0 < S; s0 += kPlanThreads) {
-    const int s = s0 + tid;
-    int f = 0;
-    if (s < S) {
-      const int c = min(max(lens[s], 0), max_c);
-      f = max(1, (c + P - 1) / P) - 1;
-    }
-    int incl = f;  // inclusive scan within the warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) warp_tot[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-      int t = lane < kPlanThreads / 32 ? warp_tot[lane] : 0;
-      int ti = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, ti, o);
-        if (lane >= o) ti += v;
-      }
-      if (lane < kPlanThreads / 32) warp_tot[lane] = ti - t;  // exclusive prefix of warp totals
-      if (lane == 31) chunk_total = ti;
-    }
-    __syncthreads();
-    const int excl = base + warp_tot[wid] + incl - f;
-    for (int part = 0; part < f; ++part)
-      for (int kh = 0; kh < Hk; ++kh)
-        items[static_cast<size_t>(excl + part) * Hk + kh] = make_int2(s, (kh << 16) | part);
-    base += chunk_total;
-    __syncthreads();
-  }
-  const size_t n_full = static_cast<size_t>(base) * Hk;
+  // Let the decode grid start its set-up now; wait for earlier work on the stream (it may have
+  // written the lengths) before reading anything.
+  pa::grid_dependency_launch();
+  pa::grid_dependency_wait();
+  __shared__ int count[kBuckets], cursor[kBuckets];
+  __shared__ int c_cache[kPlanCache];
+  const int tid = threadIdx.x;
+  const int nb = min(P / kTileTokens, kBuckets);
+  for (int b = tid; b < kBuckets; b += kPlanThreads) count[b] = 0;
+  __syncthreads();
   bool clamped = false;
   for (int s = tid; s < S; s += kPlanThreads) {
-    clamped |= lens[s] > max_c;
-    const int c = min(max(lens[s], 0), max_c);
-    const int last = max(1, (c + P - 1) / P) - 1;
-    for (int kh = 0; kh < Hk; ++kh) items[n_full + static_cast<size_t>(s) * Hk + kh] = make_int2(s, (kh << 16) | last);
+    const int raw = lens[s];
+    clamped |= raw > max_c;
+    const int c = min(max(raw, 0), max_c);
+    if (s < kPlanCache) c_cache[s] = c;
+    const int f = max(1, (c + P - 1) / P) - 1;  // whole partitions before the last one
+    if (f > 0) atomicAdd(&count[nb - 1], f * Hk);
+    atomicAdd(&count[tile_bucket(c - f * P, P)], Hk);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int b = nb - 1; b >= 0; --b) {
+      cursor[b] = run;
+      run += count[b];
+    }
+    hdr[kHdrCounter] = 0;
+    hdr[kHdrNumItems] = run;
+  }
+  __syncthreads();
+  for (int s = tid; s < S; s += kPlanThreads) {
+    const int c = s < kPlanCache ? c_cache[s] : min(max(lens[s], 0), max_c);
+    const int f = max(1, (c + P - 1) / P) - 1;
+    if (f > 0) {
+      const int base = atomicAdd(&cursor[nb - 1], f * Hk);
+      for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+    }
+    const int base = atomicAdd(&cursor[tile_bucket(c - f * P, P)], Hk);
+    for (int kh = 0; kh < Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | f);
   }
   const int any_clamped = __syncthreads_or(clamped);
-  if (tid == 0) {
-    hdr[kHdrCounter] = 0;
-    hdr[kHdrNumItems] = static_cast<int>(n_full) + S * Hk;
-    hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
-  }
+  if (tid == 0) hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
 }
 
 // ---- the decode kernel --------------------------------------------------------------------------
@@ -557,6 +563,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     pa::fence_barrier_init();
   }
   __syncthreads();
+  // The plan kernel (and everything before it on the stream) must be complete from here on.
+  pa::grid_dependency_wait();
 
   if (warp == kConsumerWarps) {
     // ================================ producer warp ==========================================
@@ -574,6 +582,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       if (lane == 0) k = atomicAdd(a.hdr + kHdrCounter, 1);
       k = __shfl_sync(0xffffffffu, k, 0);
       if (k >= n_items) {
+        if (lane == 0) pa::grid_dependency_launch();  // the combine grid may start launching
         if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
         if (lane == 0) {
           meta[stage].flags = kDone;
@@ -957,6 +966,7 @@ __global__ void __launch_bounds__(256) combine_kernel(OutT* __restrict__ out, co
                                                       const int32_t* __restrict__ lens, int S, int H,
                                                       int max_parts, int P, int min_parts) {
   // Partitions past max_parts are never read: a length that needs more is cut to max_parts * P.
+  pa::grid_dependency_wait();  // launched right behind the decode grid: its partials must be complete
   constexpr int PER = D / 32;
   const long long gw = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -986,19 +996,31 @@ __global__ void __launch_bounds__(256) combine_kernel(OutT* __restrict__ out, co
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float den = 0.f;
   if (mx != -INFINITY) {
-    for (int p = 0; p < np; ++p) {
-      const float mp = pm[p];
-      if (mp == -INFINITY) continue;
-      const float w = expf(mp - mx);
-      den = fmaf(w, pl[p], den);
-      const float* src = part_o + (gw * max_parts + p) * D + lane * PER;
+    // 32 partitions at a time: lane j computes partition (base + j)'s weight, then every lane
+    // accumulates its dims over the 32 with independent loads in flight.
+    for (int base = 0; base < np; base += 32) {
+      const int p = base + lane;
+      float w = 0.f;
+      if (p < np) {
+        const float mp = pm[p];
+        w = mp == -INFINITY ? 0.f : expf(mp - mx);
+        den = fmaf(w, pl[p], den);
+      }
+      const int cnt = min(32, np - base);
+      const float* src = part_o + (gw * max_parts + base) * D + lane * PER;
+#pragma unroll 8
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
 #pragma unroll
-      for (int e = 0; e < PER; e += 2) {
-        const float2 v = *reinterpret_cast<const float2*>(src + e);
-        acc[e] = fmaf(w, v.x, acc[e]);
-        acc[e + 1] = fmaf(w, v.y, acc[e + 1]);
+        for (int e = 0; e < PER; e += 2) {
+          const float2 v = *reinterpret_cast<const float2*>(src + static_cast<size_t>(j) * D + e);
+          acc[e] = fmaf(wj, v.x, acc[e]);
+          acc[e + 1] = fmaf(wj, v.y, acc[e + 1]);
+        }
       }
     }
+#pragma unroll
+    for (int msk = 16; msk >= 1; msk >>= 1) den += __shfl_xor_sync(0xffffffffu, den, msk);
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
@@ -1006,22 +1028,7 @@ __global__ void __launch_bounds__(256) combine_kernel(OutT* __restrict__ out, co
   pa::store_pairs<OutT, PER>(o, res);
 }
 
-template <int D>
-cudaError_t launch_combine(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
-                           const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
-                           cudaStream_t st) {
-  const long long threads = static_cast<long long>(S) * H * 32;
-  const int grid = static_cast<int>((threads + 255) / 256);
-  if (grid == 0) return cudaSuccess;
-  if (out_dtype == PA_F32)
-    combine_kernel<float, D><<<grid, 256, 0, st>>>(static_cast<float*>(out), po, pm, pl, lens, S, H, max_parts, P, min_parts);
-  else if (out_dtype == PA_F16)
-    combine_kernel<__half, D><<<grid, 256, 0, st>>>(static_cast<__half*>(out), po, pm, pl, lens, S, H, max_parts, P, min_parts);
-  else
-    combine_kernel<__nv_bfloat16, D><<<grid, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), po, pm, pl, lens, S, H, max_parts, P,
-                                                           min_parts);
-  return cudaGetLastError();
-}
+
 
 // ---- host side ----------------------------------------------------------------------------------
 
@@ -1055,6 +1062,40 @@ bool make_cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialisation: the grid may start while the previous kernel on
+// the stream finishes; the kernel itself waits (griddepcontrol.wait) before touching its inputs.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <int D>
+cudaError_t launch_combine(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
+                           const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
+                           cudaStream_t st) {
+  const long long threads = static_cast<long long>(S) * H * 32;
+  const dim3 grid(static_cast<unsigned>((threads + 255) / 256)), block(256);
+  if (grid.x == 0) return cudaSuccess;
+  if (out_dtype == PA_F32)
+    return launch_pdl(combine_kernel<float, D>, grid, block, 0, st, static_cast<float*>(out), po, pm, pl, lens, S, H,
+                      max_parts, P, min_parts);
+  if (out_dtype == PA_F16)
+    return launch_pdl(combine_kernel<__half, D>, grid, block, 0, st, static_cast<__half*>(out), po, pm, pl, lens, S,
+                      H, max_parts, P, min_parts);
+  return launch_pdl(combine_kernel<__nv_bfloat16, D>, grid, block, 0, st, static_cast<__nv_bfloat16*>(out), po, pm,
+                    pl, lens, S, H, max_parts, P, min_parts);
+}
+
 struct DeviceInfo {
   int sms = 0;
 };
@@ -1086,8 +1127,8 @@ cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const De
   long long grid = static_cast<long long>(di.sms) * occupancy;
   if (grid > max_units) grid = max_units;
   if (grid < 1) grid = 1;
-  decode_kernel<T, D, G, kMma><<<static_cast<int>(grid), kThreads, C::kSmemBytes, st>>>(tk, tv, a);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<T, D, G, kMma>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::kSmemBytes,
+                    st, tk, tv, a);
 }
 
 // Tensor-core consumers for 16-bit caches unless PA_DECODE_CONSUMER=cuda_core; fp32 caches always
@@ -1123,11 +1164,13 @@ cudaError_t dispatch_16bit(int d, int g, const CUtensorMap& tk, const CUtensorMa
 }
 
 int default_partition(int S, int Hk, int max_context_len) {
-  // Whole 512-token partitions keep the partial-state traffic small (under 2% of the KV bytes
-  // at d = 128); with few (sequence, kv head) pairs, shorter partitions give every SM work.
-  const long long units512 = static_cast<long long>(S) * Hk * ((max_context_len + 511) / 512);
-  if (units512 >= 4 * 148) return 512;
-  return 256;
+  // Longer partitions mean fewer partial states to write and merge; the longest-first unit order
+  // keeps the persistent grid balanced as long as there are several units per CTA.  Measured on
+  // B200 (gqa8k_bf16, long_bf16): 1024 beats 512 and 256 by 5-15 %.
+  const long long pairs = static_cast<long long>(S) * Hk;
+  for (int P : {1024, 512, 256})
+    if (pairs * ((max_context_len + P - 1) / P) >= 4 * 148) return P;
+  return 128;
 }
 
 int max_parts_for(int max_context_len, int P) {
@@ -1219,8 +1262,8 @@ extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query,
   a.max_parts = max_parts;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  plan_kernel<<<1, kPlanThreads, 0, st>>>(context_lens, S, Hk, P, max_context_len, reinterpret_cast<int2*>(ws + wl.items), a.hdr);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, context_lens, S, Hk, P,
+                             max_context_len, reinterpret_cast<int2*>(ws + wl.items), a.hdr);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: plan launch failed: %s", cudaGetErrorString(e));
 
   const long long units = static_cast<long long>(S) * Hk * max_parts;

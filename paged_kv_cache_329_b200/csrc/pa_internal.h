@@ -17,4 +17,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : 2; }
 inline bool valid_dtype(int t) { return t == PA_F32 || t == PA_F16 || t == PA_BF16; }
 
+// pa_copy_blocks whose pair count is read on the device from *n_pairs_dev (clamped to max_pairs);
+// the grid is sized for max_pairs so the launch can be captured once and replayed.
+pa_status copy_blocks_counted(void* k_cache, void* v_cache, const int32_t* pairs, const int32_t* n_pairs_dev,
+                              int max_pairs, int Hk, int d, int B, int n_blocks, pa_dtype dtype, void* stream);
+
 }  // namespace pa

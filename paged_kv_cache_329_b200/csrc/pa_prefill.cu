@@ -1,0 +1,580 @@
+// Paged attention for several query tokens per sequence: chunked prefill, and batches that mix
+// prefill chunks with decode tokens.
+//
+// What is computed: sequence s has n_s query tokens, the last n_s of its c_s context tokens
+// (already written to the cache); the token at position p attends causally to positions 0..p,
+// o = softmax(scale * q K[0..p]^T) V[0..p] -- the decode definition ("PagedAttention原理",
+// "为什么会有 KV cache", eq. o_t; "实现一个虚拟内存", eqs. A_ij, o_i) per query token.  Prefill
+// processes a prompt's tokens together ("vllm" 2.1 Prefill); batching prefill and decode tokens of
+// different requests, with only attention aware of each token's request and phase, is Orca's
+// selective batching ("Paged Attention&Orca Paper笔记与解读").  Decode is n_s = 1.
+//
+// Design: a work unit is (sequence, kv head, 64 query rows), a row being one (token, head) pair of
+// the head group, so a unit covers 64/g tokens and all g heads that share the kv head.  One
+// producer warp streams the unit's key range [0, last position] in 64-token tiles with 2-D TMA loads
+// (the same tensor maps as decode); four consumer warps own 16 rows each and run
+// S = Q K^T and O += P V on tensor cores (mma.sync m16n8k16, fp32 accumulators), P fed back as a
+// 16-bit hi + lo pair, with the online softmax per row in fp32.  Causal masking compares each
+// key's position with the row's own position.  Every warp finishes its rows alone, so there is
+// no cross-warp merge; units are listed longest key range first.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <mutex>
+#include <utility>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace {
+
+constexpr int kTile = 64;     // key tokens per stage
+constexpr int kCW = 4;        // consumer warps
+constexpr int kThreads = (kCW + 1) * 32;
+constexpr int kRows = kCW * 16;  // query rows per unit
+constexpr int kPlanThreads = 1024;
+constexpr int kBuckets = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kHdrCounter = 0, kHdrNumItems = 1, kHdrError = 2;
+constexpr size_t kHdrBytes = 256;
+
+enum : int { kFirst = 1, kLast = 2, kDone = 4 };
+
+struct __align__(16) Meta {
+  int s, kh, q_row0, qpos0, nq, tile_pos, ntok, flags;
+};
+
+struct Args {
+  const void* q;
+  void* out;
+  int out_dtype;
+  const int32_t* q_start;
+  const int32_t* bt;
+  const int32_t* lens;
+  int S, H, Hk, max_blocks, n_blocks, B, max_c, max_q, QT;
+  float scale_log2;
+  const int2* items;
+  int* hdr;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int tokens_per_unit(int g) { return kRows / g; }
+
+size_t max_units(int S, int Hk, int g, int max_q_len) {
+  const int QT = tokens_per_unit(g);
+  return static_cast<size_t>(S) * Hk * static_cast<size_t>((max_q_len + QT - 1) / QT);
+}
+
+// Length of query chunk and context of sequence s, checked: 0 <= n <= min(c, max_q), c <= max_c.
+// Out-of-range values are cut to the bounds (and reported), so no index leaves its buffer.
+__device__ __forceinline__ void seq_sizes(const Args& a, int s, int& n, int& c, bool& bad) {
+  n = a.q_start[s + 1] - a.q_start[s];
+  c = a.lens[s];
+  bad = n < 0 || c > a.max_c || n > c || n > a.max_q;
+  c = min(max(c, 0), a.max_c);
+  n = min(min(max(n, 0), c), a.max_q);
+}
+
+__device__ __forceinline__ int bucket_of(int kv_end, int max_c) {
+  const int tiles = (kv_end + kTile - 1) / kTile, max_tiles = max(1, (max_c + kTile - 1) / kTile);
+  const int nb = min(max_tiles, kBuckets);
+  return tiles <= 1 ? 0 : min(nb - 1, ((tiles - 1) * nb) / max_tiles);
+}
+
+// Units (s, kh, q-tile), longest key range first (64 buckets of key tiles, atomic cursors).
+__global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(Args a, int2* __restrict__ items) {
+  pa::grid_dependency_launch();
+  pa::grid_dependency_wait();
+  __shared__ int count[kBuckets], cursor[kBuckets];
+  const int tid = threadIdx.x;
+  const int max_tiles = max(1, (a.max_c + kTile - 1) / kTile), nb = min(max_tiles, kBuckets);
+  for (int b = tid; b < kBuckets; b += kPlanThreads) count[b] = 0;
+  __syncthreads();
+  bool bad_any = false;
+  for (int s = tid; s < a.S; s += kPlanThreads) {
+    int n, c;
+    bool bad;
+    seq_sizes(a, s, n, c, bad);
+    bad_any |= bad;
+    for (int t0 = 0; t0 < n; t0 += a.QT) atomicAdd(&count[bucket_of(c - n + min(t0 + a.QT, n), a.max_c)], a.Hk);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int b = nb - 1; b >= 0; --b) {
+      cursor[b] = run;
+      run += count[b];
+    }
+    a.hdr[kHdrCounter] = 0;
+    a.hdr[kHdrNumItems] = run;
+  }
+  __syncthreads();
+  for (int s = tid; s < a.S; s += kPlanThreads) {
+    int n, c;
+    bool bad;
+    seq_sizes(a, s, n, c, bad);
+    for (int t0 = 0, qt = 0; t0 < n; t0 += a.QT, ++qt) {
+      const int base = atomicAdd(&cursor[bucket_of(c - n + min(t0 + a.QT, n), a.max_c)], a.Hk);
+      for (int kh = 0; kh < a.Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | qt);
+    }
+  }
+  const int any = __syncthreads_or(bad_any);
+  if (tid == 0) a.hdr[kHdrError] = any ? pa::kErrBadLength : 0;
+}
+
+template <int D>
+struct PCfg {
+  static constexpr int kNPanel = D / 64;  // 128-byte panels of 16-bit elements
+  static constexpr int kPanelBytes = kTile * 128;
+  static constexpr int kKVBytes = kNPanel * kPanelBytes;
+  static constexpr int kStageBytes = 2 * kKVBytes;
+  static constexpr int kStages = kNPanel == 1 ? 6 : 3;
+  static constexpr int kOffMeta = kStages * kStageBytes;
+  static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
+  static constexpr int kSmemBytes = kOffBar + 2 * kStages * 8 + 1024;
+};
+
+template <class OutT>
+__device__ __forceinline__ void store_pair(OutT* p, float x0, float x1) {
+  if constexpr (sizeof(OutT) == 4) {
+    *reinterpret_cast<float2*>(p) = make_float2(x0, x1);
+  } else {
+    OutT t[2] = {pa::from_float<OutT>(x0), pa::from_float<OutT>(x1)};
+    *reinterpret_cast<uint32_t*>(p) = *reinterpret_cast<const uint32_t*>(t);
+  }
+}
+
+template <class T, int D, int G>
+__global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                           const __grid_constant__ CUtensorMap tmV, const Args a) {
+  using C = PCfg<D>;
+  using M = pa::Mma<T>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::kStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      pa::mbar_init(&full[i], 1);
+      pa::mbar_init(&empty[i], kCW);
+    }
+    pa::fence_barrier_init();
+  }
+  __syncthreads();
+  pa::grid_dependency_wait();
+
+  if (warp == kCW) {
+    // ================================ producer warp ==========================================
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    const int n_items = a.hdr[kHdrNumItems];
+    bool ok = true;
+    while (ok) {
+      int k = 0;
+      if (lane == 0) k = atomicAdd(a.hdr + kHdrCounter, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      if (k >= n_items) {
+        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        if (lane == 0) {
+          meta[stage].flags = kDone;
+          pa::mbar_arrive(&full[stage]);
+        }
+        break;
+      }
+      const int2 it = a.items[k];
+      const int s = it.x, kh = it.y >> 16, qt = it.y & 0xffff;
+      int n, c;
+      bool bad;
+      seq_sizes(a, s, n, c, bad);
+      const int tok0 = qt * a.QT, tok1 = min(tok0 + a.QT, n);
+      const int kv_end = c - n + tok1;  // keys 0 .. kv_end-1
+      const int ntiles = max(1, (kv_end + kTile - 1) / kTile);
+      const int32_t* bt_row = a.bt + static_cast<size_t>(s) * a.max_blocks;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+        const int pos0 = tile * kTile;
+        const int ntok = max(0, min(kTile, kv_end - pos0));
+        const int nblk = (ntok + a.B - 1) / a.B;
+        const int j0 = pos0 / a.B;
+        int phys = -1;
+        if (lane < nblk) {
+          phys = __ldg(bt_row + j0 + lane);
+          if (phys < 0 || phys >= a.n_blocks) {
+            atomicOr(a.hdr + kHdrError, pa::kErrBadBlock);
+            phys = -1;
+          }
+        }
+        if (lane == 0) {
+          Meta m;
+          m.s = s;
+          m.kh = kh;
+          m.q_row0 = a.q_start[s] + tok0;
+          m.qpos0 = c - n + tok0;
+          m.nq = tok1 - tok0;
+          m.tile_pos = pos0;
+          m.ntok = ntok;
+          m.flags = (tile == 0 ? kFirst : 0) | (tile == ntiles - 1 ? kLast : 0);
+          meta[stage] = m;
+          pa::mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nblk) * a.B * D * 2u * 2u);
+        }
+        __syncwarp();
+        uint8_t* kdst = smem + stage * C::kStageBytes;
+        uint8_t* vdst = kdst + C::kKVBytes;
+        if (lane < nblk) {
+          const int y = (phys * a.Hk + kh) * a.B;
+#pragma unroll
+          for (int p = 0; p < C::kNPanel; ++p) {
+            pa::tma_load_2d(kdst + p * C::kPanelBytes + lane * a.B * 128, &tmK, p * 64, y, &full[stage]);
+            pa::tma_load_2d(vdst + p * C::kPanelBytes + lane * a.B * 128, &tmV, p * 64, y, &full[stage]);
+          }
+        }
+        ++issued;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      int st = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < C::kStages && i < issued; ++i) {
+        if (--st < 0) {
+          st = C::kStages - 1;
+          ph ^= 1;
+        }
+        pa::mbar_wait(&full[st], ph);
+      }
+    }
+    return;
+  }
+
+  // ================================== consumer warps ============================================
+  constexpr int KS = D / 16;  // k-steps of q.k
+  constexpr int DN = D / 8;   // 8-wide dim tiles of the output
+  const int gq = lane >> 2, tq = lane & 3;
+  // this thread's two rows (r, r + 8) of the warp's 16; row = token * G + head
+  const int ra = warp * 16 + gq, rb = ra + 8;
+  const int tok_a = ra / G, h_a = ra % G, tok_b = rb / G, h_b = rb % G;
+  uint32_t aq[KS][4];
+  float o[DN][4];
+  float m_run[2], l_run[2];
+  int qpos_a = 0, qpos_b = 0, row_a = -1, row_b = -1, warp_qmax = -1;
+  const int ld_tok = ((lane >> 4) << 3) + (lane & 7), ld_hi = (lane >> 3) & 1;   // K: (tok 0-7|8-15) x (lo|hi)
+  const int ldv_tok = (((lane >> 3) & 1) << 3) + (lane & 7), ldv_hi = lane >> 4;  // V: (tok lo|hi) x (dim c|c+1)
+
+  int stage = 0;
+  uint32_t phase = 0;
+  while (true) {
+    if (!pa::mbar_wait(&full[stage], phase)) {
+      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      return;
+    }
+    const Meta mt = meta[stage];
+    if (mt.flags & kDone) break;
+    const uint8_t* ks = smem + stage * C::kStageBytes;
+    const uint8_t* vs = ks + C::kKVBytes;
+
+    if (mt.flags & kFirst) {
+      const bool va = tok_a < mt.nq, vb = tok_b < mt.nq;
+      qpos_a = mt.qpos0 + tok_a;
+      qpos_b = mt.qpos0 + tok_b;
+      row_a = va ? (mt.q_row0 + tok_a) * a.H + mt.kh * G + h_a : -1;
+      row_b = vb ? (mt.q_row0 + tok_b) * a.H + mt.kh * G + h_b : -1;
+      warp_qmax = -1;
+      if (warp * 16 / G < mt.nq) warp_qmax = mt.qpos0 + min(mt.nq - 1, (warp * 16 + 15) / G);
+      const uint32_t* q32 = static_cast<const uint32_t*>(a.q);
+#pragma unroll
+      for (int k = 0; k < KS; ++k) {
+        const int col = k * 16 + 2 * tq;
+        aq[k][0] = va ? __ldg(q32 + ((static_cast<size_t>(row_a) * D + col) >> 1)) : 0u;
+        aq[k][1] = vb ? __ldg(q32 + ((static_cast<size_t>(row_b) * D + col) >> 1)) : 0u;
+        aq[k][2] = va ? __ldg(q32 + ((static_cast<size_t>(row_a) * D + col + 8) >> 1)) : 0u;
+        aq[k][3] = vb ? __ldg(q32 + ((static_cast<size_t>(row_b) * D + col + 8) >> 1)) : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < DN; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
+    }
+
+    // skip tiles wholly after this warp's last query position (or warps with no rows)
+    if (warp_qmax >= mt.tile_pos && mt.ntok > 0) {
+      // ---- S = Q K^T for 16 rows x 64 keys ----
+      float sacc[8][4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
+      const uint32_t kbase = pa::smem_addr(ks);
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          const int row = np * 16 + ld_tok, c = 2 * k + ld_hi;
+          uint32_t bf[4];
+          pa::ldsm_x4(bf, kbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          M::run(sacc[2 * np], aq[k], b0);
+          M::run(sacc[2 * np + 1], aq[k], b1);
+        }
+      // ---- causal mask, online softmax (rows a: e = 0,1; b: e = 2,3) ----
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int t = j * 8 + 2 * tq + (e & 1);
+          const int kp = mt.tile_pos + t;
+          const bool ok = t < mt.ntok && kp <= ((e < 2) ? qpos_a : qpos_b) && ((e < 2) ? row_a : row_b) >= 0;
+          sacc[j][e] = ok ? sacc[j][e] * a.scale_log2 : -INFINITY;
+          mx[e >> 1] = fmaxf(mx[e >> 1], sacc[j][e]);
+        }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+      }
+      float alpha[2], mn[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mn[r] = fmaxf(m_run[r], mx[r]);
+        alpha[r] = (mn[r] == -INFINITY) ? 1.f : exp2f(m_run[r] - mn[r]);
+        m_run[r] = mn[r];
+        l_run[r] *= alpha[r];
+      }
+#pragma unroll
+      for (int i = 0; i < DN; ++i) {
+        o[i][0] *= alpha[0];
+        o[i][1] *= alpha[0];
+        o[i][2] *= alpha[1];
+        o[i][3] *= alpha[1];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float mr = mn[e >> 1];
+          sacc[j][e] = mr == -INFINITY ? 0.f : exp2f(sacc[j][e] - mr);
+          l_run[e >> 1] += sacc[j][e];
+        }
+      // ---- O += P V, P as a 16-bit hi + lo pair ----
+      const bool partial = mt.ntok < kTile;
+      const uint32_t vbase = pa::smem_addr(vs);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t ph[4], pl[4];
+        float r0, r1, d0, d1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float* src = sacc[2 * kk + (q >> 1)] + (q & 1) * 2;  // a0: row a lo toks, a1: row b, a2/a3: hi toks
+          ph[q] = M::pack(src[0], src[1], r0, r1);
+          pl[q] = M::pack(src[0] - r0, src[1] - r1, d0, d1);
+        }
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+        if (partial) {
+          const int t0 = kk * 16 + 2 * tq;
+          mlo = (t0 < mt.ntok ? 0x0000ffffu : 0u) | (t0 + 1 < mt.ntok ? 0xffff0000u : 0u);
+          mhi = (t0 + 8 < mt.ntok ? 0x0000ffffu : 0u) | (t0 + 9 < mt.ntok ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int dn = 0; dn < DN; dn += 2) {
+          const int row = kk * 16 + ldv_tok, c = dn + ldv_hi;
+          uint32_t vf[4];
+          pa::ldsm_x4_trans(vf, vbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+          const uint32_t b0[2] = {vf[0] & mlo, vf[1] & mhi}, b1[2] = {vf[2] & mlo, vf[3] & mhi};
+          M::run(o[dn], ph, b0);
+          M::run(o[dn], pl, b0);
+          M::run(o[dn + 1], ph, b1);
+          M::run(o[dn + 1], pl, b1);
+        }
+      }
+    }
+
+    __syncwarp();
+    if (lane == 0) pa::mbar_arrive(&empty[stage]);
+
+    if (mt.flags & kLast) {
+      float l[2] = {l_run[0], l_run[1]};
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+      }
+      const float inv_a = l[0] > 0.f ? 1.f / l[0] : 0.f, inv_b = l[1] > 0.f ? 1.f / l[1] : 0.f;
+#pragma unroll
+      for (int dn = 0; dn < DN; ++dn) {
+        const int col = dn * 8 + 2 * tq;
+        if (a.out_dtype == PA_F32) {
+          if (row_a >= 0) store_pair(static_cast<float*>(a.out) + static_cast<size_t>(row_a) * D + col, o[dn][0] * inv_a, o[dn][1] * inv_a);
+          if (row_b >= 0) store_pair(static_cast<float*>(a.out) + static_cast<size_t>(row_b) * D + col, o[dn][2] * inv_b, o[dn][3] * inv_b);
+        } else if (a.out_dtype == PA_F16) {
+          if (row_a >= 0) store_pair(static_cast<__half*>(a.out) + static_cast<size_t>(row_a) * D + col, o[dn][0] * inv_a, o[dn][1] * inv_a);
+          if (row_b >= 0) store_pair(static_cast<__half*>(a.out) + static_cast<size_t>(row_b) * D + col, o[dn][2] * inv_b, o[dn][3] * inv_b);
+        } else {
+          if (row_a >= 0) store_pair(static_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(row_a) * D + col, o[dn][0] * inv_a, o[dn][1] * inv_a);
+          if (row_b >= 0) store_pair(static_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(row_b) * D + col, o[dn][2] * inv_b, o[dn][3] * inv_b);
+        }
+      }
+    }
+    if (++stage == C::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+}
+
+// ---- host side ----------------------------------------------------------------------------------
+
+template <class... KArgs, class... Args2>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args2&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args2>(args)...);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long long rows, int B) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(B)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class T, int D, int G>
+cudaError_t launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
+  using C = PCfg<D>;
+  static int occupancy = -1;
+  if (occupancy < 0) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prefill_kernel<T, D, G>, kThreads, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    occupancy = occ < 1 ? 1 : occ;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long grid = static_cast<long long>(sms) * occupancy;
+  if (grid > units) grid = units;
+  if (grid < 1) grid = 1;
+  return launch_pdl(prefill_kernel<T, D, G>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::kSmemBytes, st,
+                    tk, tv, a);
+}
+
+template <class T, int D>
+cudaError_t dispatch(int g, const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
+  switch (g) {
+    case 1: return launch<T, D, 1>(tk, tv, a, units, st);
+    case 2: return launch<T, D, 2>(tk, tv, a, units, st);
+    case 4: return launch<T, D, 4>(tk, tv, a, units, st);
+    default: return launch<T, D, 8>(tk, tv, a, units, st);
+  }
+}
+
+}  // namespace
+
+extern "C" size_t pa_prefill_workspace_size(int S, int H, int Hk, int max_q_len) {
+  if (S < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || max_q_len < 0) return 0;
+  return align_up(kHdrBytes + sizeof(int2) * max_units(S, Hk, H / Hk, max_q_len), 256);
+}
+
+extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
+                                const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int S, int H, int Hk, int d, int B, int n_blocks,
+                                int max_blocks_per_seq, int max_context_len, int max_q_len, float scale,
+                                pa_dtype kv_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (S < 0 || H <= 0 || Hk <= 0 || n_blocks <= 0 || max_blocks_per_seq < 0 || max_context_len < 0 || max_q_len < 0)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: bad sizes");
+  if (H % Hk != 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: H (%d) must be a multiple of Hk (%d)", H, Hk);
+  const int g = H / Hk;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return pa::fail(PA_ERR_UNSUPPORTED, "pa_prefill: H/Hk = %d not in {1,2,4,8}", g);
+  if (d != 64 && d != 128) return pa::fail(PA_ERR_UNSUPPORTED, "pa_prefill: d = %d not in {64,128}", d);
+  if (B != 8 && B != 16 && B != 32) return pa::fail(PA_ERR_UNSUPPORTED, "pa_prefill: B = %d not in {8,16,32}", B);
+  if (kv_dtype != PA_F16 && kv_dtype != PA_BF16) return pa::fail(PA_ERR_UNSUPPORTED, "pa_prefill: caches must be fp16 or bf16");
+  if (!pa::valid_dtype(out_dtype)) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: unknown output type");
+  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: scale must be finite");
+  if (static_cast<long long>(max_blocks_per_seq) * B < max_context_len)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: max_blocks_per_seq * B < max_context_len");
+  const long long rows = static_cast<long long>(n_blocks) * Hk * B;
+  const long long units = static_cast<long long>(max_units(S, Hk, g, max_q_len));
+  if (rows >= (1ll << 31) || units >= (1ll << 30) || (max_q_len + tokens_per_unit(g) - 1) / tokens_per_unit(g) > 0xffff)
+    return pa::fail(PA_ERR_UNSUPPORTED, "pa_prefill: problem too large for 32-bit indices");
+  if (S == 0 || max_q_len == 0) return pa::ok();
+  if (!out || !query || !q_start || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: null pointer");
+  if (!pa::aligned16(out) || !pa::aligned16(query) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: workspace must be 256-byte aligned");
+  const size_t need = pa_prefill_workspace_size(S, H, Hk, max_q_len);
+  if (workspace_bytes < need) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: workspace of %zu bytes < %zu needed", workspace_bytes, need);
+  CUtensorMap tk, tv;
+  if (!cache_map(&tk, k_cache, kv_dtype, d, rows, B) || !cache_map(&tv, v_cache, kv_dtype, d, rows, B))
+    return pa::fail(PA_ERR_CUDA, "pa_prefill: could not encode the cache tensor maps");
+  Args a;
+  a.q = query;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.q_start = q_start;
+  a.bt = block_tables;
+  a.lens = context_lens;
+  a.S = S;
+  a.H = H;
+  a.Hk = Hk;
+  a.max_blocks = max_blocks_per_seq;
+  a.n_blocks = n_blocks;
+  a.B = B;
+  a.max_c = max_context_len;
+  a.max_q = max_q_len;
+  a.QT = tokens_per_unit(g);
+  a.scale_log2 = scale * kLog2e;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.hdr = reinterpret_cast<int*>(ws);
+  a.items = reinterpret_cast<const int2*>(ws + kHdrBytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pdl(prefill_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, a,
+                             reinterpret_cast<int2*>(ws + kHdrBytes));
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: plan launch failed: %s", cudaGetErrorString(e));
+  if (kv_dtype == PA_F16)
+    e = d == 64 ? dispatch<__half, 64>(g, tk, tv, a, units, st) : dispatch<__half, 128>(g, tk, tv, a, units, st);
+  else
+    e = d == 64 ? dispatch<__nv_bfloat16, 64>(g, tk, tv, a, units, st)
+                : dispatch<__nv_bfloat16, 128>(g, tk, tv, a, units, st);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s", cudaGetErrorString(e));
+  return pa::ok();
+}

@@ -1,0 +1,137 @@
+// A decode step captured once as a CUDA graph and replayed (pa_step_* in pa.h).
+//
+// The step is the serving loop's unit of work on the pages' cache ("vllm" 2.2 Decode: every step
+// appends the new token's K,V and attends over the cache; "PagedAttention原理", "解决COW": shared
+// blocks are copied before they are written): host->device copies of the step's inputs, the
+// copy-on-write block copies, the slot-mapped write, the paged decode, and the device->host copy
+// of the output.  Replaying one graph replaces a dozen stream operations per step.
+#include <cuda_runtime.h>
+
+#include <new>
+
+#include "pa_internal.h"
+
+struct pa_step {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  pa_step_desc desc;
+};
+
+namespace {
+
+bool pinned(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost;
+}
+
+pa_status record(const pa_step_desc& d, cudaStream_t s) {
+  const size_t es = pa::elem_size(d.kv_dtype), eo = pa::elem_size(d.out_dtype);
+  const size_t q_bytes = static_cast<size_t>(d.S) * d.H * d.d * es;
+  const size_t kv_bytes = static_cast<size_t>(d.S) * d.Hk * d.d * es;
+  const size_t tbl_bytes = static_cast<size_t>(d.S) * d.max_blocks_per_seq * sizeof(int32_t);
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  } h2d[] = {
+      {d.d_query, d.h_query, q_bytes},
+      {d.d_key, d.h_key, kv_bytes},
+      {d.d_value, d.h_value, kv_bytes},
+      {d.d_slots, d.h_slots, static_cast<size_t>(d.S) * sizeof(int64_t)},
+      {d.d_pairs, d.h_pairs, static_cast<size_t>(d.max_pairs) * 2 * sizeof(int32_t)},
+      {d.d_pairs + 2 * static_cast<size_t>(d.max_pairs), d.h_n_pairs, sizeof(int32_t)},
+      {d.d_tables, d.h_tables, tbl_bytes},
+      {d.d_lens, d.h_lens, static_cast<size_t>(d.S) * sizeof(int32_t)},
+  };
+  for (const Copy& c : h2d) {
+    if (c.bytes == 0) continue;
+    const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_create: capture of a copy failed: %s", cudaGetErrorString(e));
+  }
+  pa_status st = pa::copy_blocks_counted(d.k_cache, d.v_cache, d.d_pairs, d.d_pairs + 2 * static_cast<size_t>(d.max_pairs),
+                                         d.max_pairs, d.Hk, d.d, d.B, d.n_blocks, d.kv_dtype, s);
+  if (st != PA_OK) return st;
+  st = pa_cache_write(d.k_cache, d.v_cache, d.d_key, d.d_value, d.d_slots, d.S, d.Hk, d.d, d.B, d.n_blocks, d.kv_dtype, s);
+  if (st != PA_OK) return st;
+  st = pa_decode(d.d_out, d.out_dtype, d.d_query, d.k_cache, d.v_cache, d.d_tables, d.d_lens, d.S, d.H, d.Hk, d.d, d.B,
+                 d.n_blocks, d.max_blocks_per_seq, d.max_context_len, d.scale, d.kv_dtype, d.partition_size,
+                 d.workspace, d.workspace_bytes, s);
+  if (st != PA_OK) return st;
+  const cudaError_t e =
+      cudaMemcpyAsync(d.h_out, d.d_out, static_cast<size_t>(d.S) * d.H * d.d * eo, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_create: capture of the output copy failed: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_step* pa_step_create(const pa_step_desc* desc) {
+  if (!desc) {
+    pa::fail(PA_ERR_INVALID_ARG, "pa_step_create: null descriptor");
+    return nullptr;
+  }
+  const pa_step_desc& d = *desc;
+  const void* host[] = {d.h_query, d.h_key, d.h_value, d.h_slots, d.h_pairs, d.h_n_pairs, d.h_tables, d.h_lens, d.h_out};
+  for (const void* p : host)
+    if (!p || !pinned(p)) {
+      pa::fail(PA_ERR_INVALID_ARG, "pa_step_create: every host buffer must be non-null pinned memory");
+      return nullptr;
+    }
+  if (d.S <= 0 || d.max_pairs < 0 || !d.d_pairs || !d.d_query || !d.d_key || !d.d_value || !d.d_slots || !d.d_tables ||
+      !d.d_lens || !d.d_out) {
+    pa::fail(PA_ERR_INVALID_ARG, "pa_step_create: bad sizes or null device buffer");
+    return nullptr;
+  }
+  pa_step* step = new (std::nothrow) pa_step;
+  if (!step) {
+    pa::fail(PA_ERR_INVALID_ARG, "pa_step_create: out of host memory");
+    return nullptr;
+  }
+  step->desc = d;
+  cudaStream_t s = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    pa::fail(PA_ERR_CUDA, "pa_step_create: %s", cudaGetErrorString(e));
+    delete step;
+    return nullptr;
+  }
+  e = cudaStreamBeginCapture(s, cudaStreamCaptureModeRelaxed);
+  pa_status st = e == cudaSuccess ? record(d, s) : pa::fail(PA_ERR_CUDA, "pa_step_create: %s", cudaGetErrorString(e));
+  cudaGraph_t graph = nullptr;
+  if (e == cudaSuccess) {
+    const cudaError_t e2 = cudaStreamEndCapture(s, &graph);  // always end the capture
+    if (st == PA_OK && e2 != cudaSuccess) st = pa::fail(PA_ERR_CUDA, "pa_step_create: %s", cudaGetErrorString(e2));
+  }
+  if (st == PA_OK) {
+    e = cudaGraphInstantiate(&step->exec, graph, 0);
+    if (e != cudaSuccess) st = pa::fail(PA_ERR_CUDA, "pa_step_create: instantiate: %s", cudaGetErrorString(e));
+  }
+  cudaStreamDestroy(s);
+  step->graph = graph;
+  if (st != PA_OK) {
+    pa_step_destroy(step);
+    return nullptr;
+  }
+  pa::ok();
+  return step;
+}
+
+extern "C" pa_status pa_step_run(pa_step* step, void* stream) {
+  if (!step || !step->exec) return pa::fail(PA_ERR_INVALID_ARG, "pa_step_run: null step");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaGraphLaunch(step->exec, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_run: %s", cudaGetErrorString(e));
+  return pa::ok();
+}
+
+extern "C" void pa_step_destroy(pa_step* step) {
+  if (!step) return;
+  if (step->exec) cudaGraphExecDestroy(step->exec);
+  if (step->graph) cudaGraphDestroy(step->graph);
+  delete step;
+}

@@ -266,3 +266,137 @@ def test_copy_blocks_bit_exact(oracle_mod, dtype):
     bits = torch.int32 if dtype == torch.float32 else torch.int16
     assert torch.equal(kd.cpu().view(bits), k_ref.view(bits))
     assert torch.equal(vd.cpu().view(bits), v_ref.view(bits))
+
+
+# ---- the captured step (pa_step_*) ------------------------------------------------------------------
+
+def test_captured_step_matches_separate_calls(oracle_mod):
+    # Shared-prefix trajectory: forks create copy-on-write pairs every step.  Each replay of the
+    # graph must equal the oracle applied to the same block manager state.
+    B, H, Hk, d, dt = 16, 32, 8, 128, torch.bfloat16
+    mgr = api.BlockManager(512, B)
+    g = W.generator(400)
+    kc = W.randn(g, (512, Hk, B, d), dt)
+    vc = W.randn(g, (512, Hk, B, d), dt)
+    roots = []
+    for r in range(4):
+        root = mgr.seq_create()
+        mgr.reserve_slots(root, 200 + 13 * r)
+        roots.append([root] + [mgr.seq_fork(root) for _ in range(3)])
+    kd, vd = kc.cuda(), vc.cuda()
+    S = 16
+    step = api.DecodeStep(kd, vd, S, H, 32, 512, out_dtype=torch.float32)
+    k_ref, v_ref = kc.clone(), vc.clone()
+    rnd = torch.Generator().manual_seed(9)
+    for it in range(3):
+        seqs = []
+        for gi, beams in enumerate(roots):
+            parents = torch.randint(0, 4, (4,), generator=rnd).tolist()
+            kids = [mgr.seq_fork(beams[p]) for p in parents]
+            for b in beams:
+                mgr.seq_free(b)
+            roots[gi] = kids
+            seqs += kids
+        slots, pairs = mgr.reserve_slots_batch(seqs, 1, step.h_slots)
+        mgr.build_block_tables(seqs, 32, step.h_tables, step.h_lens)
+        step.set_pairs(pairs)
+        step.h_query.copy_(W.randn(g, (S, H, d), dt))
+        step.h_key.copy_(W.randn(g, (S, Hk, d), dt))
+        step.h_value.copy_(W.randn(g, (S, Hk, d), dt))
+        out = step.run().clone()
+        k_ref, v_ref = oracle_mod.copy_blocks(k_ref, v_ref, pairs)
+        k_ref, v_ref = oracle_mod.cache_write(k_ref, v_ref, step.h_key, step.h_value, step.h_slots)
+        ref = oracle_mod.decode(step.h_query, k_ref, v_ref, step.h_tables, step.h_lens)
+        assert pairs.shape[0] > 0 or it > 0
+        _assert_close(out, ref, dt, f"captured step {it}")
+    assert torch.equal(kd.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(vd.cpu().view(torch.int16), v_ref.view(torch.int16))
+    assert api.workspace_error(step.workspace) == 0
+
+
+# ---- swap to pinned host memory and back (pa_swap_blocks) --------------------------------------------
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_swap_out_and_in_bit_exact(oracle_mod, dtype):
+    n_dev, n_host, Hk, B, d = 48, 20, 8, 16, 128
+    g = W.generator(500)
+    dev_k = W.randn(g, (n_dev, Hk, B, d), dtype)
+    dev_v = W.randn(g, (n_dev, Hk, B, d), dtype)
+    host_k = W.randn(g, (n_host, Hk, B, d), dtype).pin_memory()
+    host_v = W.randn(g, (n_host, Hk, B, d), dtype).pin_memory()
+    out_pairs = torch.tensor([[3, 0], [17, 9], [40, 19], [8, 4]], dtype=torch.int32)
+    ref_hk, ref_hv = oracle_mod.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs)
+    dk, dv = dev_k.cuda(), dev_v.cuda()
+    api.pa_swap_blocks(host_k, host_v, dk, dv, out_pairs.cuda())          # device -> pinned host
+    torch.cuda.synchronize()
+    bits = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(host_k.view(bits), ref_hk.view(bits)) and torch.equal(host_v.view(bits), ref_hv.view(bits))
+    in_pairs = torch.tensor([[0, 30], [9, 31], [19, 5], [4, 47]], dtype=torch.int32).pin_memory()
+    ref_dk, ref_dv = oracle_mod.swap_blocks(dev_k, dev_v, ref_hk, ref_hv, in_pairs)
+    api.pa_swap_blocks(dk, dv, host_k, host_v, in_pairs)                  # pinned host -> device
+    torch.cuda.synchronize()
+    assert torch.equal(dk.cpu().view(bits), ref_dk.view(bits)) and torch.equal(dv.cpu().view(bits), ref_dv.view(bits))
+
+
+# ---- prefill chunks and mixed batches (pa_prefill) ---------------------------------------------------
+
+def _prefill_case(ctx, nq, H, Hk, d, B, dtype, seed):
+    case = W.paged_case("prefill", ctx, H, Hk, d, B, dtype, seed)
+    q_start = torch.tensor([0] + list(torch.tensor(nq).cumsum(0)), dtype=torch.int32)
+    q = W.randn(W.generator(seed + 7), (int(q_start[-1]), H, d), dtype)
+    return case, q, q_start
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_prefill_mixed_batch(oracle_mod, dtype, g, d, B):
+    # decode rows (n = 1), short and long chunks, chunks starting mid-context and whole prompts
+    ctx = [1, 40, 77, 200, 300, 513, 64]
+    nq = [1, 1, 77, 17, 129, 70, 64]
+    Hk = 2
+    case, q, q_start = _prefill_case(ctx, nq, g * Hk, Hk, d, B, dtype, 600 + g + d + B)
+    ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                             case.scale, n_threads=0)
+    dev = case.to("cuda")
+    ws = torch.empty(api._native.load().pa_prefill_workspace_size(case.S, case.H, Hk, max(nq)), dtype=torch.uint8,
+                     device="cuda")
+    out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                         max_context_len=max(ctx), max_q_len=max(nq), scale=case.scale, out_dtype=torch.float32,
+                         workspace=ws)
+    torch.cuda.synchronize()
+    assert api.workspace_error(ws) == 0
+    _assert_close(out.cpu(), ref, dtype, f"prefill {dtype} g={g} d={d} B={B}")
+
+
+def test_prefill_single_tokens_match_decode():
+    case = W.gqa8k_bf16(S=32)
+    dev = case.to("cuda")
+    q_start = torch.arange(case.S + 1, dtype=torch.int32, device="cuda")
+    max_c = int(case.context_lens.max())
+    out_p = api.pa_prefill(dev.q, q_start, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                           max_context_len=max_c, max_q_len=1, out_dtype=torch.float32)
+    out_d = api.pa_decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                          max_context_len=max_c, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert (out_p - out_d).abs().max().item() < 2e-3
+
+
+def test_prefill_long_prompt_sampled(oracle_mod):
+    # one 2048-token prompt chunk at the end of a 6000-token context, GQA 32/8, bf16
+    ctx, nq = [6000, 3000], [2048, 1]
+    case, q, q_start = _prefill_case(ctx, nq, 32, 8, 128, 16, torch.bfloat16, 650)
+    dev = case.to("cuda")
+    out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                         max_context_len=6000, max_q_len=2048, scale=case.scale, out_dtype=torch.float32).cpu()
+    rows = torch.tensor([0, 1, 63, 64, 1000, 2046, 2047, 2048])
+    # oracle on the sampled rows: cut each row's context at its position and decode it
+    for r in rows.tolist():
+        s = 0 if r < 2048 else 1
+        pos = ctx[s] - nq[s] + (r - int(q_start[s]))
+        lens = case.context_lens.clone()
+        lens[s] = pos + 1
+        ref = oracle_mod.decode(q[r:r + 1].expand(2, -1, -1).contiguous(), case.k_cache, case.v_cache,
+                                case.block_tables, lens, case.scale)[s]
+        _assert_close(out[r], ref, torch.bfloat16, f"prefill row {r}")

@@ -34,6 +34,12 @@ MUTANTS = [
      "o[i] += w * load_elem(k_cache, kv_dtype, rows[t - t0] * d + i);"),
     ("cache write: block and offset swapped", "const int64_t blk = slot / B, off = slot % B;",
      "const int64_t blk = slot % B, off = slot / B;"),
+    ("prefill: causal limit off by one (no self-attention)", "t <= pos", "t < pos"),
+    ("prefill: query position taken from the chunk start", "const int pos = c - n + (row - q_start[s]);",
+     "const int pos = c - n;"),
+    ("swap: source and destination pools swapped",
+     "std::memcpy(static_cast<char*>(dst_k) + dst * bytes, static_cast<const char*>(src_k) + src * bytes, bytes);",
+     "std::memcpy(static_cast<char*>(dst_k) + dst * bytes, static_cast<const char*>(src_k) + dst * bytes, bytes);"),
     ("copy: value cache not copied",
      "std::memcpy(static_cast<char*>(v_cache) + dst * bytes, static_cast<const char*>(v_cache) + src * bytes, bytes);",
      "(void)0;"),
@@ -52,6 +58,9 @@ PINS = [
     lambda o: pins.test_partition_merge_equals_plain(o, 96),
     lambda o: pins.test_cache_write_matches_index_put(o, torch.bfloat16),
     lambda o: pins.test_copy_blocks_matches_index_copy(o, torch.bfloat16),
+    lambda o: pins.test_swap_blocks_matches_index_copy(o, torch.bfloat16),
+    lambda o: pins.test_prefill_identity_table_equals_causal_sdpa(o, torch.bfloat16, 4, 128, 16),
+    lambda o: pins.test_prefill_single_token_equals_decode(o),
 ]
 
 

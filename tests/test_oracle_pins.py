@@ -280,3 +280,74 @@ def test_copy_blocks_matches_index_copy(oracle_mod, dtype):
     assert torch.equal(k2, kr) and torch.equal(v2, vr)
     # the source blocks are untouched ("解决COW": the shared block stays as it was)
     assert torch.equal(k2[1], kc[1]) and torch.equal(k2[3], kc[3])
+
+
+@pytest.mark.parametrize("dtype", DT)
+def test_swap_blocks_matches_index_copy(oracle_mod, dtype):
+    # "PagedAttention原理", 抢占与恢复 (swap): blocks move between the GPU pool and a CPU pool.
+    Hk, B, d = 2, 8, 64
+    g = torch.Generator().manual_seed(5)
+    dev_k = torch.randn(10, Hk, B, d, generator=g).to(dtype)
+    dev_v = torch.randn(10, Hk, B, d, generator=g).to(dtype)
+    host_k = torch.randn(6, Hk, B, d, generator=g).to(dtype)
+    host_v = torch.randn(6, Hk, B, d, generator=g).to(dtype)
+    out_pairs = torch.tensor([[7, 0], [2, 5], [9, 3]], dtype=torch.int32)   # device -> host
+    hk, hv = oracle_mod.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs)
+    rk, rv = host_k.clone(), host_v.clone()
+    rk[out_pairs[:, 1].long()] = dev_k[out_pairs[:, 0].long()]
+    rv[out_pairs[:, 1].long()] = dev_v[out_pairs[:, 0].long()]
+    assert torch.equal(hk, rk) and torch.equal(hv, rv)
+    in_pairs = torch.tensor([[0, 1], [5, 4], [3, 8]], dtype=torch.int32)    # host -> device, new ids
+    dk, dv = oracle_mod.swap_blocks(dev_k, dev_v, hk, hv, in_pairs)
+    assert torch.equal(dk[1], dev_k[7]) and torch.equal(dk[4], dev_k[2]) and torch.equal(dv[8], dev_v[9])
+    with pytest.raises(ValueError):
+        oracle_mod.swap_blocks(dev_k, dev_v, hk, hv, torch.tensor([[6, 0]], dtype=torch.int32))
+
+
+# ---- prefill / mixed batches (causal, several query tokens per sequence) ----------------------------
+
+@pytest.mark.parametrize("dtype,g,d,B", [(torch.float32, 1, 64, 16), (torch.bfloat16, 4, 128, 16),
+                                         (torch.float16, 8, 128, 8)])
+def test_prefill_identity_table_equals_causal_sdpa(oracle_mod, dtype, g, d, B):
+    # Contiguous blocks, the whole context as the query chunk: causal attention over the prompt.
+    torch.manual_seed(1)
+    Hk, H = 2, 2 * g
+    lens = [1, 7, B + 5, 3 * B]
+    nbs = [(c + B - 1) // B for c in lens]
+    kc = torch.randn(sum(nbs), Hk, B, d).to(dtype)
+    vc = torch.randn(sum(nbs), Hk, B, d).to(dtype)
+    bt = torch.full((len(lens), max(nbs)), -1, dtype=torch.int32)
+    pos = 0
+    for s, nb in enumerate(nbs):
+        bt[s, :nb] = torch.arange(pos, pos + nb, dtype=torch.int32)
+        pos += nb
+    q_start = torch.tensor([0] + list(torch.tensor(lens).cumsum(0)), dtype=torch.int32)
+    q = torch.randn(int(q_start[-1]), H, d).to(dtype)
+    o = oracle_mod.prefill(q, q_start, kc, vc, bt, torch.tensor(lens, dtype=torch.int32))
+    for s, c in enumerate(lens):
+        blocks = bt[s, : nbs[s]].long()
+        K = kc[blocks].permute(1, 0, 2, 3).reshape(Hk, -1, d)[:, :c].double()
+        V = vc[blocks].permute(1, 0, 2, 3).reshape(Hk, -1, d)[:, :c].double()
+        qs = q[q_start[s]: q_start[s + 1]].double().permute(1, 0, 2)        # [H, c, d]
+        ref = torch.nn.functional.scaled_dot_product_attention(qs, K, V, is_causal=True, enable_gqa=True)
+        assert torch.allclose(o[q_start[s]: q_start[s + 1]], ref.permute(1, 0, 2), atol=1e-12, rtol=1e-12)
+
+
+def test_prefill_single_token_equals_decode(oracle_mod):
+    # Decode is the n_s = 1 case: a mixed batch of decode rows and prefill chunks must agree with
+    # the decode definition on its decode rows, and on each chunk's last row.
+    case = W.paged_case("mix", [40, 130, 1, 77], 8, 2, 64, 16, torch.bfloat16, 22)
+    n = [1, 17, 1, 5]
+    q_start = torch.tensor([0] + list(torch.tensor(n).cumsum(0)), dtype=torch.int32)
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(int(q_start[-1]), 8, 64, generator=g).to(torch.bfloat16)
+    o = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens)
+    last_rows = (q_start[1:] - 1).long()
+    od = oracle_mod.decode(q[last_rows], case.k_cache, case.v_cache, case.block_tables, case.context_lens)
+    assert torch.allclose(o[last_rows], od, atol=1e-13, rtol=0)
+    # an earlier chunk row equals decode with the context cut at its position
+    lens2 = case.context_lens.clone()
+    lens2[1] = 130 - 17 + 3 + 1
+    od2 = oracle_mod.decode(q[q_start[1] + 3: q_start[1] + 4].expand(4, -1, -1).contiguous(), case.k_cache,
+                            case.v_cache, case.block_tables, lens2)
+    assert torch.allclose(o[q_start[1] + 3], od2[1], atol=1e-13, rtol=0)
