@@ -166,16 +166,12 @@ class SharedPrefixWorkload(Workload):
 
     def host_step(self, slots=None, pairs=None, tables=None, lens=None):
         # every beam picks a parent among its request's beams; children share the parent's blocks
-        i = 0
-        for r, beams in enumerate(self.groups):
-            parents = torch.randint(0, self.WIDTH, (self.WIDTH,), generator=self.rnd).tolist()
-            kids = [self.mgr.seq_fork(beams[p]) for p in parents]
-            for b in beams:
-                self.mgr.seq_free(b)
-            self.groups[r] = kids
-            for k in kids:
-                self.seqs[i] = k
-                i += 1
+        beams = self.seqs.view(self.REQUESTS, self.WIDTH)
+        choice = torch.randint(0, self.WIDTH, (self.REQUESTS, self.WIDTH), generator=self.rnd)
+        parents = torch.gather(beams, 1, choice).reshape(-1).to(torch.int32)
+        kids = self.mgr.seq_fork_batch(parents)
+        self.mgr.seq_free_batch(self.seqs)
+        self.seqs.copy_(kids)
         return super().host_step(slots, pairs, tables, lens)
 
     def unique_kv_bytes(self, tables, lens):
@@ -648,6 +644,65 @@ def run_prefill(args, rank, world, local_rank):
             "clocks": clock_info, "gpu_launches": 2 * args.steps}
 
 
+def run_cache_ops(args, rank, world, local_rank):
+    """The copy-on-write copy and the slot-mapped write at sizes where they are bandwidth-bound:
+    1024 (src, dst) pairs of gqa8k-shaped blocks (8 kv heads x 16 tokens x 128 dims, bf16) and
+    65536 new tokens written through a random slot mapping into a 65536-block pool."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    n_blocks, Hk, B, d, dt = 65536, 8, 16, 128, torch.bfloat16
+    gen = torch.Generator(device=dev).manual_seed(31 + rank)
+    kc = torch.randn((n_blocks, Hk, B, d), generator=gen, device=dev).to(dt)
+    vc = torch.randn((n_blocks, Hk, B, d), generator=gen, device=dev).to(dt)
+    g = torch.Generator().manual_seed(32)
+    perm = torch.randperm(n_blocks, generator=g)
+    pairs = torch.stack([perm[:1024], perm[1024:2048]], 1).to(torch.int32).to(dev)
+    T = 65536
+    slots = torch.randperm(n_blocks * B, generator=g)[:T].to(dev)
+    key = torch.randn((T, Hk, d), generator=gen, device=dev).to(dt)
+    val = torch.randn((T, Hk, d), generator=gen, device=dev).to(dt)
+    copy_bytes = 1024 * 2 * (Hk * B * d * 2) * 2
+    write_bytes = 2 * (T * Hk * d * 2 * 2) + 8 * T
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(args.warmup):
+        api.pa_copy_blocks(kc, vc, pairs)
+        api.pa_cache_write(kc, vc, key, val, slots)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    t0 = time.time()
+    ev[0].record()
+    for _ in range(args.steps):
+        api.pa_copy_blocks(kc, vc, pairs)
+    ev[1].record()
+    for _ in range(args.steps):
+        api.pa_cache_write(kc, vc, key, val, slots)
+    ev[2].record()
+    torch.cuda.synchronize()
+    clocks.mark(t0, time.time())
+    copy_ms, write_ms = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])
+    clock_info = clocks.finish()
+    copy_ms, write_ms = reduce_max([copy_ms, write_ms], world, dev)
+    if rank != 0:
+        return None
+    peak, kind = load_peaks()
+    copy_gbs = aggregate_value(copy_bytes, args.steps, world, copy_ms)
+    write_gbs = aggregate_value(write_bytes, args.steps, world, write_ms)
+    value = aggregate_value(copy_bytes + write_bytes, args.steps, world, copy_ms + write_ms)
+    return {"metric": "COW block copy + slot-mapped cache write effective GB/s", "value": round(value, 2),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round((copy_ms + write_ms) / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "1024 COW pairs of 8x16x128 bf16 blocks + 65536 slot writes (8x128 bf16 K and V)",
+                       "copy_bytes": copy_bytes, "write_bytes": write_bytes},
+            "kernels": {"copy_blocks": {"GB/s": round(copy_gbs, 2), "frac": round(copy_gbs / world / peak, 4),
+                                        "ms": round(copy_ms / args.steps, 5)},
+                        "cache_write": {"GB/s": round(write_gbs, 2), "frac": round(write_gbs / world / peak, 4),
+                                        "ms": round(write_ms / args.steps, 5)}},
+            "roofline": {"bound": "hbm", "achieved": round(value / world, 2), "peak": peak, "peak_kind": kind,
+                         "unit": "GB/s", "frac": round(value / world / peak, 4), "traffic": None},
+            "clocks": clock_info, "gpu_launches": 2 * args.steps}
+
+
 def run_reference(args, rank, world):
     """The oracle timed on the host cores, one bounded sample of the workload per step."""
     if rank != 0:
@@ -721,7 +776,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
-    ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS) + ["swap_bf16", "prefill_mixed_bf16"])
+    ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS) + ["swap_bf16", "prefill_mixed_bf16", "cache_ops_bf16"])
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--partition", type=int, default=0, help="decode partition size in tokens (0 = library default)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -741,7 +796,7 @@ def main():
             torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     try:
-        if args.impl == "reference" and args.workload in ("swap_bf16", "prefill_mixed_bf16"):
+        if args.impl == "reference" and args.workload in ("swap_bf16", "prefill_mixed_bf16", "cache_ops_bf16"):
             line = {"impl": "reference", "unavailable": "the oracle arm times the decode workloads only"} if rank == 0 else None
         elif args.impl == "reference":
             line = run_reference(args, rank, world)
@@ -749,6 +804,8 @@ def main():
             line = run_swap(args, rank, world, local_rank)
         elif args.workload == "prefill_mixed_bf16":
             line = run_prefill(args, rank, world, local_rank)
+        elif args.workload == "cache_ops_bf16":
+            line = run_cache_ops(args, rank, world, local_rank)
         else:
             from paged_kv_cache_329_b200 import build
 

@@ -316,6 +316,13 @@ int pa_alloc_num_free(const pa_alloc* a);
 pa_status pa_seq_create(pa_alloc* a, int32_t* seq_id);
 pa_status pa_seq_fork(pa_alloc* a, int32_t parent, int32_t* child);
 pa_status pa_seq_free(pa_alloc* a, int32_t seq_id);
+/* Batched forms for a serving step (beam search re-parenting): fork each of parents[0..n) in
+ * order (children[i] receives the new id; a parent may appear several times), or free each of
+ * seq_ids[0..n) in order.  They stop at the first unknown id and return its status; the forks or
+ * frees before it stay done. */
+pa_status pa_seq_fork_batch(pa_alloc* a, const int32_t* parents, int n, int32_t* children);
+pa_status pa_seq_free_batch(pa_alloc* a, const int32_t* seq_ids, int n);
+
 /* Length (tokens) of a sequence, or -1 if unknown. */
 int pa_seq_len(const pa_alloc* a, int32_t seq_id);
 

@@ -60,6 +60,8 @@ SIGNATURES = {
     "pa_seq_create": (I, [P, I32P]),
     "pa_seq_fork": (I, [P, ctypes.c_int32, I32P]),
     "pa_seq_free": (I, [P, ctypes.c_int32]),
+    "pa_seq_fork_batch": (I, [P, I32P, I, I32P]),
+    "pa_seq_free_batch": (I, [P, I32P, I]),
     "pa_seq_len": (I, [P, ctypes.c_int32]),
     "pa_seq_num_blocks": (I, [P, ctypes.c_int32]),
     "pa_seq_reserve_slots": (I, [P, ctypes.c_int32, I, I64P, I32P, IP]),

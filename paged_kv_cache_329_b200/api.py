@@ -292,6 +292,19 @@ class BlockManager:
     def seq_free(self, sid: int):
         _check(self._lib.pa_seq_free(self._h, sid))
 
+    def seq_fork_batch(self, parents):
+        """Fork each parent in order; returns the children as an int32 tensor."""
+        p = parents if isinstance(parents, torch.Tensor) else torch.tensor(list(parents), dtype=torch.int32)
+        kids = torch.empty(p.numel(), dtype=torch.int32)
+        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
+        _check(self._lib.pa_seq_fork_batch(self._h, i32(p), p.numel(), i32(kids)))
+        return kids
+
+    def seq_free_batch(self, seq_ids):
+        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
+        _check(self._lib.pa_seq_free_batch(self._h, ctypes.cast(ids.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+                                           ids.numel()))
+
     def seq_len(self, sid: int) -> int:
         return self._lib.pa_seq_len(self._h, sid)
 

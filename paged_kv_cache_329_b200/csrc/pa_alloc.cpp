@@ -122,6 +122,25 @@ pa_status pa_seq_free(pa_alloc* a, int32_t seq_id) {
   return pa::ok();
 }
 
+pa_status pa_seq_fork_batch(pa_alloc* a, const int32_t* parents, int n, int32_t* children) {
+  if (!a || n < 0 || (n > 0 && (!parents || !children)))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_fork_batch: bad arguments");
+  for (int i = 0; i < n; ++i) {
+    const pa_status st = pa_seq_fork(a, parents[i], children + i);
+    if (st != PA_OK) return st;
+  }
+  return pa::ok();
+}
+
+pa_status pa_seq_free_batch(pa_alloc* a, const int32_t* seq_ids, int n) {
+  if (!a || n < 0 || (n > 0 && !seq_ids)) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_free_batch: bad arguments");
+  for (int i = 0; i < n; ++i) {
+    const pa_status st = pa_seq_free(a, seq_ids[i]);
+    if (st != PA_OK) return st;
+  }
+  return pa::ok();
+}
+
 int pa_seq_len(const pa_alloc* a, int32_t seq_id) {
   if (!a) return -1;
   auto it = a->seqs.find(seq_id);

@@ -9,10 +9,11 @@
 // different requests, with only attention aware of each token's request and phase, is Orca's
 // selective batching ("Paged Attention&Orca Paper笔记与解读").  Decode is n_s = 1.
 //
-// Design: a work unit is (sequence, kv head, 64 query rows), a row being one (token, head) pair of
-// the head group, so a unit covers 64/g tokens and all g heads that share the kv head.  One
+// Design: a work unit is (sequence, kv head, 112 query rows), a row being one (token, head) pair of
+// the head group, so a unit covers 112/g tokens and all g heads that share the kv head.  One
 // producer warp streams the unit's key range [0, last position] in 64-token tiles with 2-D TMA loads
-// (the same tensor maps as decode); four consumer warps own 16 rows each and run
+// (the same tensor maps as decode); seven consumer warps own 16 rows each (their query rows staged
+// once per unit in shared memory) and run
 // S = Q K^T and O += P V on tensor cores (mma.sync m16n8k16, fp32 accumulators), P fed back as a
 // 16-bit hi + lo pair, with the online softmax per row in fp32.  Causal masking compares each
 // key's position with the row's own position.  Every warp finishes its rows alone, so there is
@@ -31,7 +32,7 @@
 namespace {
 
 constexpr int kTile = 64;     // key tokens per stage
-constexpr int kCW = 4;        // consumer warps
+constexpr int kCW = 7;        // consumer warps (with the producer: 8 warps, 256 threads)
 constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kRows = kCW * 16;  // query rows per unit
 constexpr int kPlanThreads = 1024;
@@ -132,7 +133,9 @@ struct PCfg {
   static constexpr int kKVBytes = kNPanel * kPanelBytes;
   static constexpr int kStageBytes = 2 * kKVBytes;
   static constexpr int kStages = kNPanel == 1 ? 6 : 3;
-  static constexpr int kOffMeta = kStages * kStageBytes;
+  static constexpr int kOffQ = kStages * kStageBytes;      // [4 warps][16 rows][D], 16-byte chunks
+  static constexpr int kQWarpBytes = 16 * D * 2;           // swizzled by row: chunk ^ (row & 7)
+  static constexpr int kOffMeta = kOffQ + kCW * kQWarpBytes;
   static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
   static constexpr int kSmemBytes = kOffBar + 2 * kStages * 8 + 1024;
 };
@@ -148,7 +151,7 @@ __device__ __forceinline__ void store_pair(OutT* p, float x0, float x1) {
 }
 
 template <class T, int D, int G>
-__global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV, const Args a) {
   using C = PCfg<D>;
   using M = pa::Mma<T>;
@@ -262,8 +265,8 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
   // this thread's two rows (r, r + 8) of the warp's 16; row = token * G + head
   const int ra = warp * 16 + gq, rb = ra + 8;
   const int tok_a = ra / G, h_a = ra % G, tok_b = rb / G, h_b = rb % G;
-  uint32_t aq[KS][4];
   float o[DN][4];
+  uint8_t* qw = smem + C::kOffQ + warp * C::kQWarpBytes;  // this warp's 16 query rows
   float m_run[2], l_run[2];
   int qpos_a = 0, qpos_b = 0, row_a = -1, row_b = -1, warp_qmax = -1;
   const int ld_tok = ((lane >> 4) << 3) + (lane & 7), ld_hi = (lane >> 3) & 1;   // K: (tok 0-7|8-15) x (lo|hi)
@@ -289,14 +292,18 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
       row_b = vb ? (mt.q_row0 + tok_b) * a.H + mt.kh * G + h_b : -1;
       warp_qmax = -1;
       if (warp * 16 / G < mt.nq) warp_qmax = mt.qpos0 + min(mt.nq - 1, (warp * 16 + 15) / G);
-      const uint32_t* q32 = static_cast<const uint32_t*>(a.q);
-#pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        const int col = k * 16 + 2 * tq;
-        aq[k][0] = va ? __ldg(q32 + ((static_cast<size_t>(row_a) * D + col) >> 1)) : 0u;
-        aq[k][1] = vb ? __ldg(q32 + ((static_cast<size_t>(row_b) * D + col) >> 1)) : 0u;
-        aq[k][2] = va ? __ldg(q32 + ((static_cast<size_t>(row_a) * D + col + 8) >> 1)) : 0u;
-        aq[k][3] = vb ? __ldg(q32 + ((static_cast<size_t>(row_b) * D + col + 8) >> 1)) : 0u;
+      // stage the warp's 16 query rows in shared memory (zeros for rows past the chunk)
+      {
+        constexpr int CH = D / 8;  // 16-byte chunks per row
+        const uint4* q16 = static_cast<const uint4*>(a.q);
+        for (int i = lane; i < 16 * CH; i += 32) {
+          const int r = i / CH, c = i % CH;
+          const int rr = warp * 16 + r, tok = rr / G;
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (tok < mt.nq) v = __ldg(q16 + (static_cast<size_t>((mt.q_row0 + tok) * a.H + mt.kh * G + rr % G) * D) / 8 + c);
+          *reinterpret_cast<uint4*>(qw + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
+        }
+        __syncwarp();
       }
 #pragma unroll
       for (int i = 0; i < DN; ++i)
@@ -315,17 +322,24 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[j][e] = 0.f;
       const uint32_t kbase = pa::smem_addr(ks);
+      const uint32_t qbase = pa::smem_addr(qw);
 #pragma unroll
-      for (int k = 0; k < KS; ++k)
+      for (int k = 0; k < KS; ++k) {
+        uint32_t aq[4];  // A fragment: (rows 0-7 | 8-15) x (dims lo | hi) of this k-step
+        {
+          const int r = ((lane >> 3) & 1) * 8 + (lane & 7), c = 2 * k + (lane >> 4);
+          pa::ldsm_x4(aq, qbase + r * (D * 2) + ((c ^ (r & 7)) << 4));
+        }
 #pragma unroll
         for (int np = 0; np < 4; ++np) {
           const int row = np * 16 + ld_tok, c = 2 * k + ld_hi;
           uint32_t bf[4];
           pa::ldsm_x4(bf, kbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
           const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
-          M::run(sacc[2 * np], aq[k], b0);
-          M::run(sacc[2 * np + 1], aq[k], b1);
+          M::run(sacc[2 * np], aq, b0);
+          M::run(sacc[2 * np + 1], aq, b1);
         }
+      }
       // ---- causal mask, online softmax (rows a: e = 0,1; b: e = 2,3) ----
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll

@@ -159,3 +159,24 @@ def test_batch_reservation_stops_at_first_failure():
     with pytest.raises(api.NoFreeBlock):
         nat.reserve_slots_batch([a, b, c], 1)   # a gets the last block, b cannot
     assert nat.seq_len(a) == 17 and nat.seq_len(b) == 16 and nat.seq_len(c) == 0
+
+
+def test_batched_fork_and_free_equal_single_calls():
+    B = 16
+    nat, mod = api.BlockManager(1024, B), BlockManagerModel(1024, B)
+    roots = []
+    for n in (40, 70, 16):
+        a, b = nat.seq_create(), mod.seq_create()
+        nat.reserve_slots(a, n)
+        mod.reserve_slots(b, n)
+        roots.append(a)
+    parents = [roots[0], roots[0], roots[2], roots[1], roots[0]]
+    kids = nat.seq_fork_batch(parents).tolist()
+    assert kids == [mod.seq_fork(p) for p in parents]
+    nat.seq_free_batch(roots)
+    for r in roots:
+        mod.seq_free(r)
+    _same_state(nat, mod)
+    with pytest.raises(api.PAError):
+        nat.seq_free_batch([kids[0], 999])
+    assert nat.seq_len(kids[0]) == -1          # freed before the unknown id stopped the batch
