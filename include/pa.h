@@ -133,6 +133,12 @@ int pa_decode_default_partition(int S, int Hk, int max_context_len);
  * wait timed out (the kernel gave up); bit 2 = a context length exceeded max_context_len (cut to it). */
 pa_status pa_workspace_error(const void* workspace, int* flags, void* stream);
 
+/* Self-test of the kernels' bounded waits: launches one CTA that waits, with the same wait the
+ * decode pipeline uses, on a barrier phase that nothing completes.  After limit_us microseconds
+ * (0 < limit_us <= 1e7) the wait gives up and the kernel writes the timeout bit (2) to *status
+ * (device int) instead of hanging; the context stays usable.  Used by the tests. */
+pa_status pa_selftest_wait_timeout(unsigned int limit_us, int* status, void* stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Log-sum-exp merge of per-partition partial states ("实现一个虚拟内存", eq. A_ij: its denominator
  * is a sum over blocks, so it can be accumulated over any partition of the blocks and merged).
@@ -240,7 +246,9 @@ pa_status pa_swap_blocks(void* dst_k, void* dst_v, int n_dst_blocks, const void*
  * into a CUDA graph over the fixed buffers named in the descriptor; pa_step_run replays it, so a
  * step costs one graph launch instead of a dozen API calls (the copy-on-write count, which varies
  * from step to step, travels in pinned memory with the other inputs).  The caller refills the host
- * buffers (e.g. with pa_seq_reserve_slots_batch and pa_build_block_tables) before each run.
+ * buffers (e.g. with pa_seq_reserve_slots_batch and pa_build_block_tables) before each run.  Host
+ * inputs that are laid out like their device buffers (same offsets from one host block and one
+ * device block, gaps up to 4 KiB) are copied with a single transfer.
  */
 typedef struct {
   /* pinned host buffers (cudaHostAlloc / cudaHostRegister memory), read or written by each run */
@@ -281,6 +289,11 @@ pa_step* pa_step_create(const pa_step_desc* desc);
 
 /* Launches the captured step on `stream` and waits for it (the output is in h_out on return). */
 pa_status pa_step_run(pa_step* step, void* stream);
+
+/* Launches the captured step on `stream` and returns at once; the output is in h_out once the
+ * stream has reached this point.  With two steps (two sets of buffers) a caller can prepare the
+ * next step's inputs on the host while the GPU runs the current one. */
+pa_status pa_step_launch(pa_step* step, void* stream);
 
 void pa_step_destroy(pa_step* step);
 

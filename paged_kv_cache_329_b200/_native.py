@@ -43,12 +43,14 @@ SIGNATURES = {
     "pa_prefill_workspace_size": (SZ, [I, I, I, I]),
     "pa_prefill": (I, [P, I, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, SZ, P]),
     "pa_workspace_error": (I, [P, IP, P]),
+    "pa_selftest_wait_timeout": (I, [ctypes.c_uint, P, P]),
     "pa_combine": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),
     "pa_cache_write": (I, [P, P, P, P, P, I, I, I, I, I, I, P]),
     "pa_copy_blocks": (I, [P, P, P, I, I, I, I, I, I, P]),
     "pa_swap_blocks": (I, [P, P, I, P, P, I, P, I, I, I, I, I, P]),
     "pa_step_create": (P, [ctypes.POINTER(StepDesc)]),
     "pa_step_run": (I, [P, P]),
+    "pa_step_launch": (I, [P, P]),
     "pa_step_destroy": (None, [P]),
     "pa_alloc_create": (P, [I, I]),
     "pa_alloc_destroy": (None, [P]),

@@ -187,24 +187,27 @@ class DecodeStep:
         dt, dev = k_cache.dtype, k_cache.device
         out_dtype = out_dtype or dt
         max_pairs = S if max_pairs is None else max_pairs
-        pin = lambda shape, t: torch.empty(shape, dtype=t).pin_memory()
-        self.h_query, self.h_key, self.h_value = pin((S, H, d), dt), pin((S, Hk, d), dt), pin((S, Hk, d), dt)
-        self.h_slots = pin((S,), torch.int64)
-        self.h_pairs = pin((max(max_pairs, 1), 2), torch.int32)
-        self.h_n_pairs = pin((1,), torch.int32)
-        self.h_tables = pin((S, max_blocks_per_seq), torch.int32)
-        self.h_lens = pin((S,), torch.int32)
-        self.h_out = pin((S, H, d), out_dtype)
-        self.h_n_pairs.zero_()
+        # Every input lives at the same offset in one pinned block and one device block, so the
+        # captured step moves them with a single host->device transfer.
+        mp = max(max_pairs, 1)
+        fields = [("query", (S, H, d), dt), ("key", (S, Hk, d), dt), ("value", (S, Hk, d), dt),
+                  ("slots", (S,), torch.int64), ("pairs", (2 * mp + 4,), torch.int32),
+                  ("tables", (S, max_blocks_per_seq), torch.int32), ("lens", (S,), torch.int32)]
+        offs, total = {}, 0
+        for name, shape, t in fields:
+            offs[name] = total
+            total += -(-math.prod(shape) * torch.empty((), dtype=t).element_size() // 256) * 256
+        self._h_block = torch.zeros(total, dtype=torch.uint8).pin_memory()
+        self._d_block = torch.zeros(total, dtype=torch.uint8, device=dev)
+        for name, shape, t in fields:
+            n = math.prod(shape) * torch.empty((), dtype=t).element_size()
+            setattr(self, "h_" + name, self._h_block[offs[name]: offs[name] + n].view(t).view(shape))
+            setattr(self, "d_" + name, self._d_block[offs[name]: offs[name] + n].view(t).view(shape))
+        self.h_n_pairs = self.h_pairs[2 * mp: 2 * mp + 1]           # the count sits right after the pairs
+        self.h_pairs = self.h_pairs[: 2 * mp].view(mp, 2)
+        self.h_out = torch.empty((S, H, d), dtype=out_dtype).pin_memory()
+        self.d_out = torch.zeros((S, H, d), dtype=out_dtype, device=dev)
         self.h_slots.fill_(-1)
-        self.h_lens.zero_()
-        dz = lambda shape, t: torch.zeros(shape, dtype=t, device=dev)
-        self.d_query, self.d_key, self.d_value = dz((S, H, d), dt), dz((S, Hk, d), dt), dz((S, Hk, d), dt)
-        self.d_slots = dz((S,), torch.int64)
-        self.d_pairs = dz((2 * max(max_pairs, 1) + 4,), torch.int32)
-        self.d_tables = dz((S, max_blocks_per_seq), torch.int32)
-        self.d_lens = dz((S,), torch.int32)
-        self.d_out = dz((S, H, d), out_dtype)
         self.workspace = alloc_workspace(S, H, Hk, d, max_context_len, partition_size, dev)
         self.k_cache, self.v_cache = k_cache, v_cache
         vp = lambda t: t.data_ptr()
@@ -219,9 +222,7 @@ class DecodeStep:
         self._h = self._lib.pa_step_create(ctypes.byref(desc))
         if not self._h:
             raise PAError(PA_ERR_INVALID_ARG, self._lib.pa_last_error().decode())
-        self.h2d_bytes = sum(t.numel() * t.element_size() for t in
-                             (self.h_query, self.h_key, self.h_value, self.h_slots, self.h_pairs, self.h_n_pairs,
-                              self.h_tables, self.h_lens))
+        self.h2d_bytes = self._h_block.numel()
         self.d2h_bytes = self.h_out.numel() * self.h_out.element_size()
 
     def set_pairs(self, pairs):
@@ -235,6 +236,10 @@ class DecodeStep:
     def run(self, stream=None):
         _check(self._lib.pa_step_run(self._h, _stream(stream)))
         return self.h_out
+
+    def launch(self, stream=None):
+        """Enqueue the step and return; h_out is valid once the stream reaches it."""
+        _check(self._lib.pa_step_launch(self._h, _stream(stream)))
 
     def __del__(self):
         h = getattr(self, "_h", None)

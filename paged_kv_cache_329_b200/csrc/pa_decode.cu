@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const DecodeArgs a) {
   using C = Cfg<T, D, G>;
-  constexpr int E = C::kE, L = C::kL, CPL = C::kCPL, NG = C::kNG, R = C::kR, AC = C::kAcc;
+  constexpr int E = C::kE, L = C::kL, CPL = C::kCPL, R = C::kR, AC = C::kAcc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -1350,4 +1350,31 @@ extern "C" pa_status pa_decode_noalloc(void* out, pa_dtype out_dtype, const void
   return pa_decode(out, out_dtype, query, k_cache, v_cache, block_tables, context_lens, S, H, Hk, d, B, n_blocks,
                    max_blocks_per_seq, max_context_len, scale, kv_dtype, partition_size, scratch,
                    kNoAllocScratchBytes, stream);
+}
+
+// ---- self-test of the bounded pipeline wait -------------------------------------------------------
+namespace {
+
+// Waits, with the same helper the decode pipeline uses, for a barrier phase that nothing completes;
+// the wait gives up after limit_ns and the kernel reports it instead of spinning.
+__global__ void wait_probe_kernel(unsigned long long limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    pa::mbar_init(&bar, 1);
+    pa::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool done = pa::mbar_wait(&bar, 0, limit_ns);
+  if (threadIdx.x == 0) *status = done ? 0 : pa::kErrWaitTimeout;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_selftest_wait_timeout(unsigned int limit_us, int* status, void* stream) {
+  if (!status || limit_us == 0 || limit_us > 10000000u)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_selftest_wait_timeout: need a status pointer and 0 < limit_us <= 1e7");
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us, status);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_selftest_wait_timeout: %s", cudaGetErrorString(e));
+  return pa::ok();
 }

@@ -23,7 +23,10 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "pa_device.cuh"
@@ -62,7 +65,7 @@ struct Args {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-int tokens_per_unit(int g) { return kRows / g; }
+int tokens_per_unit(int g) { return kRows / g; }  // the smaller of the two unit sizes
 
 size_t max_units(int S, int Hk, int g, int max_q_len) {
   const int QT = tokens_per_unit(g);
@@ -74,7 +77,8 @@ size_t max_units(int S, int Hk, int g, int max_q_len) {
 __device__ __forceinline__ void seq_sizes(const Args& a, int s, int& n, int& c, bool& bad) {
   n = a.q_start[s + 1] - a.q_start[s];
   c = a.lens[s];
-  bad = n < 0 || c > a.max_c || n > c || n > a.max_q;
+  bad = n < 0 || c > a.max_c || n > c || n > a.max_q || a.q_start[s] < 0;
+  if (a.q_start[s] < 0) n = 0;  // a negative row offset would index below the query buffer
   c = min(max(c, 0), a.max_c);
   n = min(min(max(n, 0), c), a.max_q);
 }
@@ -150,6 +154,97 @@ __device__ __forceinline__ void store_pair(OutT* p, float x0, float x1) {
   }
 }
 
+// The producer warp: pulls units, streams each unit's causal key range [0, last position] in
+// 64-token tiles (one 2-D TMA box per block and 128-byte panel, for K and for V) into the stage
+// ring, with the unit's geometry in the stage's Meta; signals kDone when the units run out.
+template <int D, class C>
+__device__ __forceinline__ void produce_units(uint8_t* smem, Meta* meta, uint64_t* full, uint64_t* empty,
+                                              const CUtensorMap& tmK, const CUtensorMap& tmV, const Args& a,
+                                              int lane) {
+  int stage = 0, issued = 0;
+  uint32_t phase = 0;
+  const int n_items = a.hdr[kHdrNumItems];
+  bool ok = true;
+  while (ok) {
+    int k = 0;
+    if (lane == 0) k = atomicAdd(a.hdr + kHdrCounter, 1);
+    k = __shfl_sync(0xffffffffu, k, 0);
+    if (k >= n_items) {
+      if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+      if (lane == 0) {
+        meta[stage].flags = kDone;
+        pa::mbar_arrive(&full[stage]);
+      }
+      break;
+    }
+    const int2 it = a.items[k];
+    const int s = it.x, kh = it.y >> 16, qt = it.y & 0xffff;
+    int n, c;
+    bool bad;
+    seq_sizes(a, s, n, c, bad);
+    const int tok0 = qt * a.QT, tok1 = min(tok0 + a.QT, n);
+    const int kv_end = c - n + tok1;  // keys 0 .. kv_end-1
+    const int ntiles = max(1, (kv_end + kTile - 1) / kTile);
+    const int32_t* bt_row = a.bt + static_cast<size_t>(s) * a.max_blocks;
+    for (int tile = 0; tile < ntiles; ++tile) {
+      if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+      const int pos0 = tile * kTile;
+      const int ntok = max(0, min(kTile, kv_end - pos0));
+      const int nblk = (ntok + a.B - 1) / a.B;
+      const int j0 = pos0 / a.B;
+      int phys = -1;
+      if (lane < nblk) {
+        phys = __ldg(bt_row + j0 + lane);
+        if (phys < 0 || phys >= a.n_blocks) {
+          atomicOr(a.hdr + kHdrError, pa::kErrBadBlock);
+          phys = -1;
+        }
+      }
+      if (lane == 0) {
+        Meta m;
+        m.s = s;
+        m.kh = kh;
+        m.q_row0 = a.q_start[s] + tok0;
+        m.qpos0 = c - n + tok0;
+        m.nq = tok1 - tok0;
+        m.tile_pos = pos0;
+        m.ntok = ntok;
+        m.flags = (tile == 0 ? kFirst : 0) | (tile == ntiles - 1 ? kLast : 0);
+        meta[stage] = m;
+        pa::mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nblk) * a.B * D * 2u * 2u);
+      }
+      __syncwarp();
+      uint8_t* kdst = smem + stage * C::kStageBytes;
+      uint8_t* vdst = kdst + C::kKVBytes;
+      if (lane < nblk) {
+        const int y = (phys * a.Hk + kh) * a.B;
+#pragma unroll
+        for (int p = 0; p < C::kNPanel; ++p) {
+          pa::tma_load_2d(kdst + p * C::kPanelBytes + lane * a.B * 128, &tmK, p * 64, y, &full[stage]);
+          pa::tma_load_2d(vdst + p * C::kPanelBytes + lane * a.B * 128, &tmV, p * 64, y, &full[stage]);
+        }
+      }
+      ++issued;
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
+  if (!ok) {
+    if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    int st = stage;
+    uint32_t ph = phase;
+    for (int i = 0; i < C::kStages && i < issued; ++i) {
+      if (--st < 0) {
+        st = C::kStages - 1;
+        ph ^= 1;
+      }
+      pa::mbar_wait(&full[st], ph);
+    }
+  }
+}
+
 template <class T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV, const Args a) {
@@ -172,89 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   pa::grid_dependency_wait();
 
   if (warp == kCW) {
-    // ================================ producer warp ==========================================
-    int stage = 0, issued = 0;
-    uint32_t phase = 0;
-    const int n_items = a.hdr[kHdrNumItems];
-    bool ok = true;
-    while (ok) {
-      int k = 0;
-      if (lane == 0) k = atomicAdd(a.hdr + kHdrCounter, 1);
-      k = __shfl_sync(0xffffffffu, k, 0);
-      if (k >= n_items) {
-        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-        if (lane == 0) {
-          meta[stage].flags = kDone;
-          pa::mbar_arrive(&full[stage]);
-        }
-        break;
-      }
-      const int2 it = a.items[k];
-      const int s = it.x, kh = it.y >> 16, qt = it.y & 0xffff;
-      int n, c;
-      bool bad;
-      seq_sizes(a, s, n, c, bad);
-      const int tok0 = qt * a.QT, tok1 = min(tok0 + a.QT, n);
-      const int kv_end = c - n + tok1;  // keys 0 .. kv_end-1
-      const int ntiles = max(1, (kv_end + kTile - 1) / kTile);
-      const int32_t* bt_row = a.bt + static_cast<size_t>(s) * a.max_blocks;
-      for (int tile = 0; tile < ntiles; ++tile) {
-        if (!pa::mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-        const int pos0 = tile * kTile;
-        const int ntok = max(0, min(kTile, kv_end - pos0));
-        const int nblk = (ntok + a.B - 1) / a.B;
-        const int j0 = pos0 / a.B;
-        int phys = -1;
-        if (lane < nblk) {
-          phys = __ldg(bt_row + j0 + lane);
-          if (phys < 0 || phys >= a.n_blocks) {
-            atomicOr(a.hdr + kHdrError, pa::kErrBadBlock);
-            phys = -1;
-          }
-        }
-        if (lane == 0) {
-          Meta m;
-          m.s = s;
-          m.kh = kh;
-          m.q_row0 = a.q_start[s] + tok0;
-          m.qpos0 = c - n + tok0;
-          m.nq = tok1 - tok0;
-          m.tile_pos = pos0;
-          m.ntok = ntok;
-          m.flags = (tile == 0 ? kFirst : 0) | (tile == ntiles - 1 ? kLast : 0);
-          meta[stage] = m;
-          pa::mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nblk) * a.B * D * 2u * 2u);
-        }
-        __syncwarp();
-        uint8_t* kdst = smem + stage * C::kStageBytes;
-        uint8_t* vdst = kdst + C::kKVBytes;
-        if (lane < nblk) {
-          const int y = (phys * a.Hk + kh) * a.B;
-#pragma unroll
-          for (int p = 0; p < C::kNPanel; ++p) {
-            pa::tma_load_2d(kdst + p * C::kPanelBytes + lane * a.B * 128, &tmK, p * 64, y, &full[stage]);
-            pa::tma_load_2d(vdst + p * C::kPanelBytes + lane * a.B * 128, &tmV, p * 64, y, &full[stage]);
-          }
-        }
-        ++issued;
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-    if (!ok) {
-      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
-      int st = stage;
-      uint32_t ph = phase;
-      for (int i = 0; i < C::kStages && i < issued; ++i) {
-        if (--st < 0) {
-          st = C::kStages - 1;
-          ph ^= 1;
-        }
-        pa::mbar_wait(&full[st], ph);
-      }
-    }
+    produce_units<D, C>(smem, meta, full, empty, tmK, tmV, a, lane);
     return;
   }
 
@@ -446,6 +459,275 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   }
 }
 
+
+
+// ---- tcgen05 consumers -------------------------------------------------------------------------------
+// 128 query rows per unit, one per TMEM lane.  Warps 0-3: one thread per row (softmax, P, output);
+// warp 4: the TMA producer; warp 5: allocates TMEM and one lane issues the MMAs.  Per 64-key tile:
+//   S[128 x 64]  = Q K^T              8 (d = 128) tcgen05.mma, A = Q tile, B = K tile (K-major)
+//   softmax rows read S from TMEM, mask causally, write P (hi and lo bf16/fp16 parts) to shared memory
+//   O[128 x d]  += P_hi V + P_lo V     8 tcgen05.mma, B = V tile (MN-major: d contiguous)
+// The running maximum is updated lazily: O (in TMEM) is rescaled only when a row's maximum grows by
+// more than 2^8, which keeps every exponent bounded and costs nothing in the common case.
+constexpr int kURows = 128;
+constexpr int kUProducer = 4, kUMma = 5;
+constexpr int kUThreads = 6 * 32;
+constexpr uint32_t kTmemCols = 256;  // S: columns 0..63, O: columns 64..64+d-1
+
+template <int D>
+struct UCfg {
+  static constexpr int kNPanel = D / 64;
+  static constexpr int kPanelBytes = kTile * 128;
+  static constexpr int kKVBytes = kNPanel * kPanelBytes;
+  static constexpr int kStageBytes = 2 * kKVBytes;
+  static constexpr int kStages = kNPanel == 1 ? 6 : 3;
+  static constexpr int kQPanelBytes = kURows * 128;
+  static constexpr int kOffQ = kStages * kStageBytes;
+  static constexpr int kOffP = kOffQ + kNPanel * kQPanelBytes;  // P hi, then P lo: [128 rows][64 keys]
+  static constexpr int kOffMeta = kOffP + 2 * kURows * 128;
+  static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
+  static constexpr int kNBars = 2 * kStages + 5;  // full, empty, q_ready, s_full, p_full, o_done, teardown
+  static constexpr int kOffTmem = kOffBar + kNBars * 8;
+  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;
+};
+
+template <class T, int D, int G>
+__global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                    const __grid_constant__ CUtensorMap tmV,
+                                                                    const Args a) {
+  using C = UCfg<D>;
+  constexpr bool kBF16 = sizeof(T) == 2 && !std::is_same<T, __half>::value;
+  constexpr uint32_t kIdescS = pa::umma_idesc(kBF16, kURows, kTile, false, false);
+  constexpr uint32_t kIdescO = pa::umma_idesc(kBF16, kURows, D, false, true);
+  constexpr int KS = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* q_ready = empty + C::kStages;
+  uint64_t* s_full = q_ready + 1;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* teardown = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      pa::mbar_init(&full[i], 1);
+      pa::mbar_init(&empty[i], 1);  // one tcgen05.commit per tile
+    }
+    pa::mbar_init(q_ready, kURows);
+    pa::mbar_init(s_full, 1);
+    pa::mbar_init(p_full, kURows);
+    pa::mbar_init(o_done, 1);
+    pa::mbar_init(teardown, kURows);
+    pa::fence_barrier_init();
+  }
+  if (warp == kUMma) {
+    pa::tmem_alloc(tmem_slot, kTmemCols);
+    pa::tmem_relinquish();
+  }
+  pa::tc_fence_before();
+  __syncthreads();
+  pa::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 64;
+  pa::grid_dependency_wait();
+
+  if (warp == kUProducer) {
+    produce_units<D, C>(smem, meta, full, empty, tmK, tmV, a, lane);
+    return;
+  }
+
+  if (warp == kUMma) {
+    // ================================ MMA issuer ==============================================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, q_ph = 0, p_ph = 0;
+      const uint32_t q_base = pa::smem_addr(smem + C::kOffQ);
+      const uint32_t p_hi = pa::smem_addr(smem + C::kOffP), p_lo = p_hi + kURows * 128;
+      bool ok = true;
+      while (true) {
+        if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+        const Meta mt = meta[stage];
+        if (mt.flags & kDone) break;
+        if (mt.flags & kFirst) {
+          if (!pa::mbar_wait(q_ready, q_ph)) { ok = false; break; }
+          q_ph ^= 1;
+        }
+        pa::tc_fence_after();
+        const uint32_t kb = pa::smem_addr(smem + stage * C::kStageBytes), vb = kb + C::kKVBytes;
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+          const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
+          const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
+          pa::umma_f16(tS, da, db, kIdescS, k > 0 ? 1u : 0u);
+        }
+        pa::umma_commit(s_full);
+        if (!pa::mbar_wait(p_full, p_ph)) { ok = false; break; }
+        p_ph ^= 1;
+        pa::tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t da = pa::sw128_desc((part ? p_lo : p_hi) + kk * 32, 16, 1024);
+            const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
+            const bool first = (mt.flags & kFirst) && part == 0 && kk == 0;
+            pa::umma_f16(tO, da, db, kIdescO, first ? 0u : 1u);
+          }
+        pa::umma_commit(o_done);
+        pa::umma_commit(&empty[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    }
+    __syncwarp();
+    // free TMEM once the row threads are done with it
+    pa::mbar_wait(teardown, 0);
+    pa::tc_fence_after();
+    pa::tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
+
+  // ================================== row threads (warps 0-3) =====================================
+  const int r = warp * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  uint8_t* qs = smem + C::kOffQ;
+  uint8_t* ph = smem + C::kOffP;
+  uint8_t* pl = ph + kURows * 128;
+  int stage = 0;
+  uint32_t phase = 0, s_ph = 0, o_ph = 0;
+  float m_used = -INFINITY, l = 0.f;
+  int row_global = -1, qpos = 0;
+  bool pv_pending = false, ok = true;
+  while (true) {
+    if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+    const Meta mt = meta[stage];
+    if (mt.flags & kDone) break;
+    if (mt.flags & kFirst) {
+      const int tok = r / G, h = r % G;
+      const bool valid = tok < mt.nq;
+      qpos = mt.qpos0 + tok;
+      row_global = valid ? (mt.q_row0 + tok) * a.H + mt.kh * G + h : -1;
+      const uint4* src = static_cast<const uint4*>(a.q) + static_cast<size_t>(valid ? row_global : 0) * (D / 8);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(qs + (c >> 3) * C::kQPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+      }
+      pa::fence_proxy_async_smem();
+      pa::mbar_arrive(q_ready);
+      m_used = -INFINITY;
+      l = 0.f;
+    }
+    // keys past the tile's valid ones get p = 0; zero their V rows, which may hold stale or unused data
+    if (mt.ntok < kTile) {
+      uint8_t* vs = smem + stage * C::kStageBytes + C::kKVBytes;
+      for (int i = r; i < (kTile - mt.ntok) * (D / 8); i += kURows) {
+        const int row = mt.ntok + i / (D / 8), c = i % (D / 8);
+        *reinterpret_cast<uint4*>(vs + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    if (!pa::mbar_wait(s_full, s_ph)) { ok = false; break; }
+    s_ph ^= 1;
+    pa::tc_fence_after();
+    float sv[kTile];
+#pragma unroll
+    for (int j = 0; j < kTile / 16; ++j) {
+      float t[16];
+      pa::tmem_ld16(tS + lane_base + 16 * j, t);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sv[16 * j + e] = t[e];
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) {
+      const bool vis = row_global >= 0 && c < mt.ntok && mt.tile_pos + c <= qpos;
+      sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, sv[c]);
+    }
+    // the previous tile's P -> O product must be complete before P is overwritten or O rescaled
+    if (pv_pending) {
+      if (!pa::mbar_wait(o_done, o_ph)) { ok = false; break; }
+      o_ph ^= 1;
+      pv_pending = false;
+      pa::tc_fence_after();
+    }
+    if (mx > m_used + 8.f) {
+      if (m_used != -INFINITY) {
+        const float f = exp2f(m_used - mx);
+        l *= f;
+        if (!(mt.flags & kFirst)) {
+#pragma unroll 1
+          for (int j = 0; j < D / 16; ++j) {
+            float t[16];
+            pa::tmem_ld16(tO + lane_base + 16 * j, t);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) t[e] *= f;
+            pa::tmem_st16(tO + lane_base + 16 * j, t);
+          }
+        }
+      }
+      m_used = mx;
+    }
+    float lsum = 0.f;
+#pragma unroll
+    for (int c8 = 0; c8 < kTile / 8; ++c8) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p0 = m_used == -INFINITY ? 0.f : exp2f(sv[8 * c8 + 2 * e] - m_used);
+        const float p1 = m_used == -INFINITY ? 0.f : exp2f(sv[8 * c8 + 2 * e + 1] - m_used);
+        lsum += p0 + p1;
+        float r0, r1, d0, d1;
+        hi[e] = pa::Mma<T>::pack(p0, p1, r0, r1);
+        lo[e] = pa::Mma<T>::pack(p0 - r0, p1 - r1, d0, d1);
+      }
+      const int off = r * 128 + ((c8 ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    l += lsum;
+    pa::fence_proxy_async_smem();
+    pa::tc_fence_before();
+    pa::mbar_arrive(p_full);
+    pv_pending = true;
+    if (mt.flags & kLast) {
+      if (!pa::mbar_wait(o_done, o_ph)) { ok = false; break; }
+      o_ph ^= 1;
+      pv_pending = false;
+      pa::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int j = 0; j < D / 16; ++j) {
+        float t[16];
+        pa::tmem_ld16(tO + lane_base + 16 * j, t);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t[e] *= inv;
+        if (row_global >= 0) {
+          const size_t off = static_cast<size_t>(row_global) * D + 16 * j;
+          if (a.out_dtype == PA_F32) pa::store_floats<float, 16>(static_cast<float*>(a.out) + off, t);
+          else if (a.out_dtype == PA_F16) pa::store_floats<__half, 16>(static_cast<__half*>(a.out) + off, t);
+          else pa::store_floats<__nv_bfloat16, 16>(static_cast<__nv_bfloat16*>(a.out) + off, t);
+        }
+      }
+    }
+    if (++stage == C::kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+  if (!ok && lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+  pa::tc_fence_before();
+  pa::mbar_arrive(teardown);
+}
+
 // ---- host side ----------------------------------------------------------------------------------
 
 template <class... KArgs, class... Args2>
@@ -511,8 +793,44 @@ cudaError_t launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, 
                     tk, tv, a);
 }
 
+template <class T, int D, int G>
+cudaError_t launch_umma(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
+  using C = UCfg<D>;
+  static bool ready = false;
+  if (!ready) {
+    const cudaError_t e = cudaFuncSetAttribute(prefill_umma_kernel<T, D, G>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    ready = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long grid = sms;  // one CTA per SM: its shared memory and TMEM allocation are sized for that
+  if (grid > units) grid = units;
+  if (grid < 1) grid = 1;
+  return launch_pdl(prefill_umma_kernel<T, D, G>, dim3(static_cast<unsigned>(grid)), dim3(kUThreads),
+                    C::kSmemBytes, st, tk, tv, a);
+}
+
+// tcgen05 consumers unless PA_PREFILL_CONSUMER=mma_sync.
+bool use_umma() {
+  const char* v = std::getenv("PA_PREFILL_CONSUMER");
+  return !(v && std::strcmp(v, "mma_sync") == 0);
+}
+
+int rows_per_unit() { return use_umma() ? kURows : kRows; }
+
 template <class T, int D>
 cudaError_t dispatch(int g, const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
+  if (use_umma()) {
+    switch (g) {
+      case 1: return launch_umma<T, D, 1>(tk, tv, a, units, st);
+      case 2: return launch_umma<T, D, 2>(tk, tv, a, units, st);
+      case 4: return launch_umma<T, D, 4>(tk, tv, a, units, st);
+      default: return launch_umma<T, D, 8>(tk, tv, a, units, st);
+    }
+  }
   switch (g) {
     case 1: return launch<T, D, 1>(tk, tv, a, units, st);
     case 2: return launch<T, D, 2>(tk, tv, a, units, st);
@@ -575,7 +893,7 @@ extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query
   a.B = B;
   a.max_c = max_context_len;
   a.max_q = max_q_len;
-  a.QT = tokens_per_unit(g);
+  a.QT = rows_per_unit() / g;  // the workspace is sized for the smaller unit (more units)
   a.scale_log2 = scale * kLog2e;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.hdr = reinterpret_cast<int*>(ws);

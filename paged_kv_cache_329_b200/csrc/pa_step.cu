@@ -7,7 +7,9 @@
 // of the output.  Replaying one graph replaces a dozen stream operations per step.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <new>
+#include <vector>
 
 #include "pa_internal.h"
 
@@ -47,8 +49,29 @@ pa_status record(const pa_step_desc& d, cudaStream_t s) {
       {d.d_tables, d.h_tables, tbl_bytes},
       {d.d_lens, d.h_lens, static_cast<size_t>(d.S) * sizeof(int32_t)},
   };
-  for (const Copy& c : h2d) {
-    if (c.bytes == 0) continue;
+  // Copies whose host and device buffers keep the same relative placement (e.g. carved from one
+  // host block and one device block with equal offsets) are merged into one transfer, gaps of at
+  // most 4 KiB included.
+  std::vector<Copy> list;
+  for (const Copy& c : h2d)
+    if (c.bytes) list.push_back(c);
+  std::sort(list.begin(), list.end(), [](const Copy& x, const Copy& y) { return x.src < y.src; });
+  std::vector<Copy> merged;
+  for (const Copy& c : list) {
+    if (!merged.empty()) {
+      Copy& m = merged.back();
+      const char* m_src = static_cast<const char*>(m.src);
+      const char* c_src = static_cast<const char*>(c.src);
+      const char* m_dst = static_cast<const char*>(m.dst);
+      const char* c_dst = static_cast<const char*>(c.dst);
+      if (c_src >= m_src + m.bytes && c_src - m_src == c_dst - m_dst && c_src - (m_src + m.bytes) <= 4096) {
+        m.bytes = static_cast<size_t>(c_src - m_src) + c.bytes;
+        continue;
+      }
+    }
+    merged.push_back(c);
+  }
+  for (const Copy& c : merged) {
     const cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_create: capture of a copy failed: %s", cudaGetErrorString(e));
   }
@@ -126,6 +149,13 @@ extern "C" pa_status pa_step_run(pa_step* step, void* stream) {
   cudaError_t e = cudaGraphLaunch(step->exec, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_run: %s", cudaGetErrorString(e));
+  return pa::ok();
+}
+
+extern "C" pa_status pa_step_launch(pa_step* step, void* stream) {
+  if (!step || !step->exec) return pa::fail(PA_ERR_INVALID_ARG, "pa_step_launch: null step");
+  const cudaError_t e = cudaGraphLaunch(step->exec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_step_launch: %s", cudaGetErrorString(e));
   return pa::ok();
 }
 

@@ -400,3 +400,36 @@ def test_prefill_long_prompt_sampled(oracle_mod):
         ref = oracle_mod.decode(q[r:r + 1].expand(2, -1, -1).contiguous(), case.k_cache, case.v_cache,
                                 case.block_tables, lens, case.scale)[s]
         _assert_close(out[r], ref, torch.bfloat16, f"prefill row {r}")
+
+
+
+# ---- failure detection without a GPU fault ------------------------------------------------------------
+
+def test_bounded_wait_gives_up_and_context_survives():
+    import time as _time
+    lib = api._native.load()
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    t0 = _time.time()
+    assert lib.pa_selftest_wait_timeout(50000, api._ptr(status), None) == api.PA_OK   # 50 ms
+    torch.cuda.synchronize()
+    assert int(status) == 2                      # the wait ran out and said so
+    assert _time.time() - t0 < 5.0
+    case = W.paged_case("after", [100, 7], 8, 2, 64, 16, torch.bfloat16, 700)
+    assert torch.isfinite(_run(case)).all()     # the context still runs kernels
+
+
+def test_out_of_range_block_id_is_reported_not_faulted(oracle_mod):
+    # A bad table entry reads as zeros (the TMA unit fills a box outside the tensor) and sets bit 0
+    # of the error word; every other sequence is unaffected.
+    case = W.paged_case("badblk", [40, 100, 33], 8, 2, 128, 16, torch.bfloat16, 701, sentinel="none")
+    bt = case.block_tables.clone()
+    bt[1, 2] = case.n_blocks + 5                 # out of range
+    dev = W.DecodeCase("badblk", case.q, case.k_cache, case.v_cache, bt, case.context_lens, case.scale,
+                       case.H, case.Hk, case.d, case.B).to("cuda")
+    ws = api.alloc_workspace(case.S, case.H, case.Hk, case.d, 100, 64)
+    out = api.pa_decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, max_context_len=100,
+                        scale=case.scale, out_dtype=torch.float32, partition_size=64, workspace=ws).cpu()
+    assert api.workspace_error(ws) & 1
+    ref = oracle_mod.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, case.scale)
+    _assert_close(out[[0, 2]], ref[[0, 2]], torch.bfloat16, "other sequences")
+    assert torch.isfinite(out[1]).all()
