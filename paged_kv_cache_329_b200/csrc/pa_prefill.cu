@@ -460,19 +460,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 }
 
 
-
 // ---- tcgen05 consumers -------------------------------------------------------------------------------
-// 128 query rows per unit, one per TMEM lane.  Warps 0-3: one thread per row (softmax, P, output);
-// warp 4: the TMA producer; warp 5: allocates TMEM and one lane issues the MMAs.  Per 64-key tile:
-//   S[128 x 64]  = Q K^T              8 (d = 128) tcgen05.mma, A = Q tile, B = K tile (K-major)
-//   softmax rows read S from TMEM, mask causally, write P (hi and lo bf16/fp16 parts) to shared memory
-//   O[128 x d]  += P_hi V + P_lo V     8 tcgen05.mma, B = V tile (MN-major: d contiguous)
-// The running maximum is updated lazily: O (in TMEM) is rescaled only when a row's maximum grows by
-// more than 2^8, which keeps every exponent bounded and costs nothing in the common case.
-constexpr int kURows = 128;
-constexpr int kUProducer = 4, kUMma = 5;
-constexpr int kUThreads = 6 * 32;
-constexpr uint32_t kTmemCols = 256;  // S: columns 0..63, O: columns 64..64+d-1
+// 256 query rows per unit in two 128-row halves A and B (one TMEM lane per row in each half).
+// Warps 0-3 own the rows of half A, warps 4-7 those of half B (softmax, P, output); warp 8 is the
+// TMA producer; warp 9 allocates TMEM and one lane issues the MMAs.  Per 64-key tile j and half h:
+//   S_h[128 x 64]  = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
+//   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) to smem
+//   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    B = V tile (MN-major: d contiguous)
+// The MMA issue order S_A(j+1) before PV_B(j) lets one half's softmax run while the tensor core
+// serves the other half.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
+// when a row's maximum grows by more than 2^8, which keeps every exponent bounded.
+constexpr int kURows = 128;                  // rows per half (TMEM lanes)
+constexpr int kUHalves = 2;
+constexpr int kUUnitRows = kURows * kUHalves;
+constexpr int kUProducer = 8, kUMma = 9;
+constexpr int kUThreads = 10 * 32;
+constexpr uint32_t kTmemCols = 512;          // S_A 0..63, S_B 64..127, O_A 128.., O_B 128+d..
 
 template <int D>
 struct UCfg {
@@ -482,13 +485,18 @@ struct UCfg {
   static constexpr int kStageBytes = 2 * kKVBytes;
   static constexpr int kStages = kNPanel == 1 ? 6 : 3;
   static constexpr int kQPanelBytes = kURows * 128;
+  static constexpr int kQHalfBytes = kNPanel * kQPanelBytes;
+  static constexpr int kPHalfBytes = 2 * kURows * 128;           // hi then lo: [128 rows][64 keys] each
   static constexpr int kOffQ = kStages * kStageBytes;
-  static constexpr int kOffP = kOffQ + kNPanel * kQPanelBytes;  // P hi, then P lo: [128 rows][64 keys]
-  static constexpr int kOffMeta = kOffP + 2 * kURows * 128;
+  static constexpr int kOffP = kOffQ + kUHalves * kQHalfBytes;
+  static constexpr int kOffMeta = kOffP + kUHalves * kPHalfBytes;
   static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
-  static constexpr int kNBars = 2 * kStages + 5;  // full, empty, q_ready, s_full, p_full, o_done, teardown
+  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done; then teardown
+  static constexpr int kNBars = 2 * kStages + 4 * kUHalves + 1;
   static constexpr int kOffTmem = kOffBar + kNBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(128 + kUHalves * D <= static_cast<int>(kTmemCols), "TMEM columns: two S tiles and two O tiles");
 };
 
 template <class T, int D, int G>
@@ -505,11 +513,11 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + C::kStages;
-  uint64_t* q_ready = empty + C::kStages;
-  uint64_t* s_full = q_ready + 1;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* teardown = o_done + 1;
+  uint64_t* q_ready = empty + C::kStages;      // [2]
+  uint64_t* s_full = q_ready + kUHalves;       // [2]
+  uint64_t* p_full = s_full + kUHalves;        // [2]
+  uint64_t* o_done = p_full + kUHalves;        // [2]
+  uint64_t* teardown = o_done + kUHalves;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -517,11 +525,13 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       pa::mbar_init(&full[i], 1);
       pa::mbar_init(&empty[i], 1);  // one tcgen05.commit per tile
     }
-    pa::mbar_init(q_ready, kURows);
-    pa::mbar_init(s_full, 1);
-    pa::mbar_init(p_full, kURows);
-    pa::mbar_init(o_done, 1);
-    pa::mbar_init(teardown, kURows);
+    for (int h = 0; h < kUHalves; ++h) {
+      pa::mbar_init(&q_ready[h], kURows);
+      pa::mbar_init(&s_full[h], 1);
+      pa::mbar_init(&p_full[h], kURows);
+      pa::mbar_init(&o_done[h], 1);
+    }
+    pa::mbar_init(teardown, kUUnitRows);
     pa::fence_barrier_init();
   }
   if (warp == kUMma) {
@@ -532,7 +542,6 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   __syncthreads();
   pa::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 64;
   pa::grid_dependency_wait();
 
   if (warp == kUProducer) {
@@ -544,44 +553,74 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     // ================================ MMA issuer ==============================================
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, q_ph = 0, p_ph = 0;
+      uint32_t phase = 0, q_ph = 0, p_ph[2] = {0, 0};
       const uint32_t q_base = pa::smem_addr(smem + C::kOffQ);
-      const uint32_t p_hi = pa::smem_addr(smem + C::kOffP), p_lo = p_hi + kURows * 128;
+      const uint32_t p_base = pa::smem_addr(smem + C::kOffP);
       bool ok = true;
-      while (true) {
-        if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
-        const Meta mt = meta[stage];
-        if (mt.flags & kDone) break;
-        if (mt.flags & kFirst) {
-          if (!pa::mbar_wait(q_ready, q_ph)) { ok = false; break; }
-          q_ph ^= 1;
-        }
-        pa::tc_fence_after();
-        const uint32_t kb = pa::smem_addr(smem + stage * C::kStageBytes), vb = kb + C::kKVBytes;
+      auto issue_s = [&](int h, int st) {
+        const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
+        const uint32_t qb = q_base + h * C::kQHalfBytes;
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
-          const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
+          const uint64_t da = pa::sw128_desc(qb + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
           const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-          pa::umma_f16(tS, da, db, kIdescS, k > 0 ? 1u : 0u);
+          pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
         }
-        pa::umma_commit(s_full);
-        if (!pa::mbar_wait(p_full, p_ph)) { ok = false; break; }
-        p_ph ^= 1;
-        pa::tc_fence_after();
+        pa::umma_commit(&s_full[h]);
+      };
+      auto issue_pv = [&](int h, int st, bool first_tile) {
+        const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
+        const uint32_t pb = p_base + h * C::kPHalfBytes;
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t da = pa::sw128_desc((part ? p_lo : p_hi) + kk * 32, 16, 1024);
+            const uint64_t da = pa::sw128_desc(pb + part * (kURows * 128) + kk * 32, 16, 1024);
             const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
-            const bool first = (mt.flags & kFirst) && part == 0 && kk == 0;
-            pa::umma_f16(tO, da, db, kIdescO, first ? 0u : 1u);
+            const bool init = first_tile && part == 0 && kk == 0;
+            pa::umma_f16(tmem + 128 + D * h, da, db, kIdescO, init ? 0u : 1u);
           }
-        pa::umma_commit(o_done);
-        pa::umma_commit(&empty[stage]);
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1;
+        pa::umma_commit(&o_done[h]);
+      };
+      while (ok) {
+        // first tile of a unit
+        if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+        Meta mt = meta[stage];
+        if (mt.flags & kDone) break;
+        if (!pa::mbar_wait(&q_ready[0], q_ph) || !pa::mbar_wait(&q_ready[1], q_ph)) { ok = false; break; }
+        q_ph ^= 1;
+        pa::tc_fence_after();
+        issue_s(0, stage);
+        issue_s(1, stage);
+        bool first = true;
+        while (true) {
+          const bool last = (mt.flags & kLast) != 0;
+          int nstage = stage + 1;
+          uint32_t nphase = phase;
+          if (nstage == C::kStages) {
+            nstage = 0;
+            nphase ^= 1;
+          }
+          if (!pa::mbar_wait(&p_full[0], p_ph[0])) { ok = false; break; }
+          p_ph[0] ^= 1;
+          pa::tc_fence_after();
+          issue_pv(0, stage, first);
+          if (!last) {
+            if (!pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
+            pa::tc_fence_after();
+            issue_s(0, nstage);
+          }
+          if (!pa::mbar_wait(&p_full[1], p_ph[1])) { ok = false; break; }
+          p_ph[1] ^= 1;
+          pa::tc_fence_after();
+          issue_pv(1, stage, first);
+          pa::umma_commit(&empty[stage]);
+          if (!last) issue_s(1, nstage);
+          stage = nstage;
+          phase = nphase;
+          if (last) break;
+          mt = meta[stage];
+          first = false;
         }
       }
       if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
@@ -594,12 +633,19 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     return;
   }
 
-  // ================================== row threads (warps 0-3) =====================================
-  const int r = warp * 32 + lane;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  uint8_t* qs = smem + C::kOffQ;
-  uint8_t* ph = smem + C::kOffP;
+  // ================================== row threads (warps 0-7) =====================================
+  const int half = warp >> 2;                         // 0: rows 0..127, 1: rows 128..255
+  const int hr = (warp & 3) * 32 + lane;              // row within the half = TMEM lane
+  const int r = half * kURows + hr;                   // row within the unit
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tS = tmem + 64 * half, tO = tmem + 128 + D * half;
+  uint8_t* qs = smem + C::kOffQ + half * C::kQHalfBytes;
+  uint8_t* ph = smem + C::kOffP + half * C::kPHalfBytes;
   uint8_t* pl = ph + kURows * 128;
+  uint64_t* my_q_ready = &q_ready[half];
+  uint64_t* my_s_full = &s_full[half];
+  uint64_t* my_p_full = &p_full[half];
+  uint64_t* my_o_done = &o_done[half];
   int stage = 0;
   uint32_t phase = 0, s_ph = 0, o_ph = 0;
   float m_used = -INFINITY, l = 0.f;
@@ -618,23 +664,24 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(qs + (c >> 3) * C::kQPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(qs + (c >> 3) * C::kQPanelBytes + hr * 128 + (((c & 7) ^ (hr & 7)) << 4)) = v;
       }
       pa::fence_proxy_async_smem();
-      pa::mbar_arrive(q_ready);
+      pa::mbar_arrive(my_q_ready);
       m_used = -INFINITY;
       l = 0.f;
     }
-    // keys past the tile's valid ones get p = 0; zero their V rows, which may hold stale or unused data
-    if (mt.ntok < kTile) {
+    // keys past the tile's valid ones get p = 0; zero their V rows, which may hold stale or unused
+    // data (half A does it: both halves' P.V products are issued after half A's P is ready)
+    if (mt.ntok < kTile && half == 0) {
       uint8_t* vs = smem + stage * C::kStageBytes + C::kKVBytes;
-      for (int i = r; i < (kTile - mt.ntok) * (D / 8); i += kURows) {
+      for (int i = hr; i < (kTile - mt.ntok) * (D / 8); i += kURows) {
         const int row = mt.ntok + i / (D / 8), c = i % (D / 8);
         *reinterpret_cast<uint4*>(vs + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
             make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    if (!pa::mbar_wait(s_full, s_ph)) { ok = false; break; }
+    if (!pa::mbar_wait(my_s_full, s_ph)) { ok = false; break; }
     s_ph ^= 1;
     pa::tc_fence_after();
     float sv[kTile];
@@ -652,9 +699,9 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
       mx = fmaxf(mx, sv[c]);
     }
-    // the previous tile's P -> O product must be complete before P is overwritten or O rescaled
+    // this half's previous P.V product must be complete before P is overwritten or O rescaled
     if (pv_pending) {
-      if (!pa::mbar_wait(o_done, o_ph)) { ok = false; break; }
+      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
       o_ph ^= 1;
       pv_pending = false;
       pa::tc_fence_after();
@@ -689,17 +736,17 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
         hi[e] = pa::Mma<T>::pack(p0, p1, r0, r1);
         lo[e] = pa::Mma<T>::pack(p0 - r0, p1 - r1, d0, d1);
       }
-      const int off = r * 128 + ((c8 ^ (r & 7)) << 4);
+      const int off = hr * 128 + ((c8 ^ (hr & 7)) << 4);
       *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
     l += lsum;
     pa::fence_proxy_async_smem();
     pa::tc_fence_before();
-    pa::mbar_arrive(p_full);
+    pa::mbar_arrive(my_p_full);
     pv_pending = true;
     if (mt.flags & kLast) {
-      if (!pa::mbar_wait(o_done, o_ph)) { ok = false; break; }
+      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
       o_ph ^= 1;
       pv_pending = false;
       pa::tc_fence_after();
@@ -819,7 +866,7 @@ bool use_umma() {
   return !(v && std::strcmp(v, "mma_sync") == 0);
 }
 
-int rows_per_unit() { return use_umma() ? kURows : kRows; }
+int rows_per_unit() { return use_umma() ? kUUnitRows : kRows; }
 
 template <class T, int D>
 cudaError_t dispatch(int g, const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
