@@ -557,29 +557,35 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       const uint32_t q_base = pa::smem_addr(smem + C::kOffQ);
       const uint32_t p_base = pa::smem_addr(smem + C::kOffP);
       bool ok = true;
-      auto issue_s = [&](int h, int st) {
-        const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
-        const uint32_t qb = q_base + h * C::kQHalfBytes;
+      // A half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
+      // MMAs, but its barriers are committed all the same so that both sides count the same phases.
+      auto issue_s = [&](int h, int st, bool active) {
+        if (active) {
+          const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
+          const uint32_t qb = q_base + h * C::kQHalfBytes;
 #pragma unroll
-        for (int k = 0; k < KS; ++k) {
-          const uint64_t da = pa::sw128_desc(qb + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
-          const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-          pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
+          for (int k = 0; k < KS; ++k) {
+            const uint64_t da = pa::sw128_desc(qb + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
+            const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
+            pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
+          }
         }
         pa::umma_commit(&s_full[h]);
       };
-      auto issue_pv = [&](int h, int st, bool first_tile) {
-        const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
-        const uint32_t pb = p_base + h * C::kPHalfBytes;
+      auto issue_pv = [&](int h, int st, bool first_tile, bool active) {
+        if (active) {
+          const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
+          const uint32_t pb = p_base + h * C::kPHalfBytes;
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+          for (int part = 0; part < 2; ++part)
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t da = pa::sw128_desc(pb + part * (kURows * 128) + kk * 32, 16, 1024);
-            const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
-            const bool init = first_tile && part == 0 && kk == 0;
-            pa::umma_f16(tmem + 128 + D * h, da, db, kIdescO, init ? 0u : 1u);
-          }
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t da = pa::sw128_desc(pb + part * (kURows * 128) + kk * 32, 16, 1024);
+              const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
+              const bool init = first_tile && part == 0 && kk == 0;
+              pa::umma_f16(tmem + 128 + D * h, da, db, kIdescO, init ? 0u : 1u);
+            }
+        }
         pa::umma_commit(&o_done[h]);
       };
       while (ok) {
@@ -590,8 +596,9 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
         if (!pa::mbar_wait(&q_ready[0], q_ph) || !pa::mbar_wait(&q_ready[1], q_ph)) { ok = false; break; }
         q_ph ^= 1;
         pa::tc_fence_after();
-        issue_s(0, stage);
-        issue_s(1, stage);
+        const bool act_b = mt.nq * G > kURows;  // half A always holds the unit's first query
+        issue_s(0, stage, true);
+        issue_s(1, stage, act_b);
         bool first = true;
         while (true) {
           const bool last = (mt.flags & kLast) != 0;
@@ -604,18 +611,18 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
           if (!pa::mbar_wait(&p_full[0], p_ph[0])) { ok = false; break; }
           p_ph[0] ^= 1;
           pa::tc_fence_after();
-          issue_pv(0, stage, first);
+          issue_pv(0, stage, first, true);
           if (!last) {
             if (!pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
             pa::tc_fence_after();
-            issue_s(0, nstage);
+            issue_s(0, nstage, true);
           }
           if (!pa::mbar_wait(&p_full[1], p_ph[1])) { ok = false; break; }
           p_ph[1] ^= 1;
           pa::tc_fence_after();
-          issue_pv(1, stage, first);
+          issue_pv(1, stage, first, act_b);
           pa::umma_commit(&empty[stage]);
-          if (!last) issue_s(1, nstage);
+          if (!last) issue_s(1, nstage, act_b);
           stage = nstage;
           phase = nphase;
           if (last) break;
@@ -637,6 +644,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   const int half = warp >> 2;                         // 0: rows 0..127, 1: rows 128..255
   const int hr = (warp & 3) * 32 + lane;              // row within the half = TMEM lane
   const int r = half * kURows + hr;                   // row within the unit
+  const int warp_row0 = half * kURows + (warp & 3) * 32;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tS = tmem + 64 * half, tO = tmem + 128 + D * half;
   uint8_t* qs = smem + C::kOffQ + half * C::kQHalfBytes;
@@ -650,7 +658,8 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   uint32_t phase = 0, s_ph = 0, o_ph = 0;
   float m_used = -INFINITY, l = 0.f;
   int row_global = -1, qpos = 0;
-  bool pv_pending = false, ok = true;
+  bool pv_pending = false, ok = true, warp_active = false;
+  const float sl2 = a.scale_log2 == 0.f ? 1.f : fabsf(a.scale_log2);
   while (true) {
     if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
     const Meta mt = meta[stage];
@@ -660,10 +669,21 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       const bool valid = tok < mt.nq;
       qpos = mt.qpos0 + tok;
       row_global = valid ? (mt.q_row0 + tok) * a.H + mt.kh * G + h : -1;
+      // a warp none of whose rows holds a query skips the arithmetic (its S, P and O are unused)
+      // but keeps to the barrier protocol
+      warp_active = mt.nq * G > warp_row0;
       const uint4* src = static_cast<const uint4*>(a.q) + static_cast<size_t>(valid ? row_global : 0) * (D / 8);
+      // the scale's sign is carried by q (exact: a sign flip, or zero for scale 0), so that the
+      // row maximum can be taken before scaling by sl2 >= 0
+      const uint32_t q_flip = a.scale_log2 < 0.f ? 0x80008000u : 0u;
+      const bool q_keep = valid && a.scale_log2 != 0.f;
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        uint4 v = q_keep ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        v.x ^= q_flip;
+        v.y ^= q_flip;
+        v.z ^= q_flip;
+        v.w ^= q_flip;
         *reinterpret_cast<uint4*>(qs + (c >> 3) * C::kQPanelBytes + hr * 128 + (((c & 7) ^ (hr & 7)) << 4)) = v;
       }
       pa::fence_proxy_async_smem();
@@ -683,34 +703,41 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     }
     if (!pa::mbar_wait(my_s_full, s_ph)) { ok = false; break; }
     s_ph ^= 1;
-    pa::tc_fence_after();
-    float sv[kTile];
-#pragma unroll
-    for (int j = 0; j < kTile / 16; ++j) {
-      float t[16];
-      pa::tmem_ld16(tS + lane_base + 16 * j, t);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sv[16 * j + e] = t[e];
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kTile; ++c) {
-      const bool vis = row_global >= 0 && c < mt.ntok && mt.tile_pos + c <= qpos;
-      sv[c] = vis ? sv[c] * a.scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sv[c]);
-    }
-    // this half's previous P.V product must be complete before P is overwritten or O rescaled
+    // S(j) is issued after this half's P.V(j-1), so that product is complete as well
     if (pv_pending) {
       if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
       o_ph ^= 1;
       pv_pending = false;
-      pa::tc_fence_after();
     }
-    if (mx > m_used + 8.f) {
-      if (m_used != -INFINITY) {
-        const float f = exp2f(m_used - mx);
-        l *= f;
-        if (!(mt.flags & kFirst)) {
+    pa::tc_fence_after();
+    if (warp_active) {
+      float sv[kTile];
+      pa::tmem_ld64(tS + lane_base, sv);
+      // causal and length masking only on tiles that reach past the unit's first query position
+      // or past the context (the same decision for the whole unit)
+      if (mt.ntok < kTile || mt.tile_pos + kTile - 1 > mt.qpos0) {
+        const int cut = row_global < 0 ? 0 : min(qpos - mt.tile_pos + 1, mt.ntok);
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) sv[c] = c < cut ? sv[c] : -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+      // tcgen05.ld/st are warp-collective, so the rescale of O is decided per warp; rows that do not
+      // need it take the factor 1
+      const bool grow = mx > m_used + 8.f;
+      if (__any_sync(0xffffffffu, grow)) {
+        float f = 1.f;
+        if (grow) {
+          if (m_used != -INFINITY) f = pa::ex2(m_used - mx);
+          l *= f;
+          m_used = mx;
+        }
+        if (!(mt.flags & kFirst) && __any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll 1
           for (int j = 0; j < D / 16; ++j) {
             float t[16];
@@ -721,27 +748,26 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
           }
         }
       }
-      m_used = mx;
-    }
-    float lsum = 0.f;
+      // p = 2^(s * sl2 - m); with no visible key so far every s is -inf and p = 0
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c8 = 0; c8 < kTile / 8; ++c8) {
-      uint32_t hi[4], lo[4];
+      for (int c8 = 0; c8 < kTile / 8; ++c8) {
+        uint32_t hi[4], lo[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p0 = m_used == -INFINITY ? 0.f : exp2f(sv[8 * c8 + 2 * e] - m_used);
-        const float p1 = m_used == -INFINITY ? 0.f : exp2f(sv[8 * c8 + 2 * e + 1] - m_used);
-        lsum += p0 + p1;
-        float r0, r1, d0, d1;
-        hi[e] = pa::Mma<T>::pack(p0, p1, r0, r1);
-        lo[e] = pa::Mma<T>::pack(p0 - r0, p1 - r1, d0, d1);
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = pa::ex2(fmaf(sv[8 * c8 + 2 * e], sl2, neg_m));
+          const float p1 = pa::ex2(fmaf(sv[8 * c8 + 2 * e + 1], sl2, neg_m));
+          ls[e] += p0 + p1;
+          pa::Split<T>::run(p0, p1, hi[e], lo[e]);
+        }
+        const int off = hr * 128 + ((c8 ^ (hr & 7)) << 4);
+        *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      const int off = hr * 128 + ((c8 ^ (hr & 7)) << 4);
-      *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      pa::fence_proxy_async_smem();
     }
-    l += lsum;
-    pa::fence_proxy_async_smem();
     pa::tc_fence_before();
     pa::mbar_arrive(my_p_full);
     pv_pending = true;
@@ -750,18 +776,20 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       o_ph ^= 1;
       pv_pending = false;
       pa::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (warp_active) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int j = 0; j < D / 16; ++j) {
-        float t[16];
-        pa::tmem_ld16(tO + lane_base + 16 * j, t);
+        for (int j = 0; j < D / 16; ++j) {
+          float t[16];
+          pa::tmem_ld16(tO + lane_base + 16 * j, t);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] *= inv;
-        if (row_global >= 0) {
-          const size_t off = static_cast<size_t>(row_global) * D + 16 * j;
-          if (a.out_dtype == PA_F32) pa::store_floats<float, 16>(static_cast<float*>(a.out) + off, t);
-          else if (a.out_dtype == PA_F16) pa::store_floats<__half, 16>(static_cast<__half*>(a.out) + off, t);
-          else pa::store_floats<__nv_bfloat16, 16>(static_cast<__nv_bfloat16*>(a.out) + off, t);
+          for (int e = 0; e < 16; ++e) t[e] *= inv;
+          if (row_global >= 0) {
+            const size_t off = static_cast<size_t>(row_global) * D + 16 * j;
+            if (a.out_dtype == PA_F32) pa::store_floats<float, 16>(static_cast<float*>(a.out) + off, t);
+            else if (a.out_dtype == PA_F16) pa::store_floats<__half, 16>(static_cast<__half*>(a.out) + off, t);
+            else pa::store_floats<__nv_bfloat16, 16>(static_cast<__nv_bfloat16*>(a.out) + off, t);
+          }
         }
       }
     }

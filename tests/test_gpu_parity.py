@@ -370,6 +370,52 @@ def test_prefill_mixed_batch(oracle_mod, dtype, g, d, B):
     _assert_close(out.cpu(), ref, dtype, f"prefill {dtype} g={g} d={d} B={B}")
 
 
+@pytest.fixture(params=["tcgen05", "mma_sync"])
+def prefill_consumer(request, monkeypatch):
+    """pa_prefill consumers: tcgen05 with TMEM accumulators (default) or mma.sync."""
+    if request.param == "mma_sync":
+        monkeypatch.setenv("PA_PREFILL_CONSUMER", "mma_sync")
+    else:
+        monkeypatch.delenv("PA_PREFILL_CONSUMER", raising=False)
+    return request.param
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("scale", [-0.3, 0.0, 0.125, 0.3, 1.0])
+def test_prefill_scale_sign(oracle_mod, prefill_consumer, dtype, scale):
+    # the softmax of scale * q.k for a negative scale (the largest weight on the smallest score),
+    # for scale 0 (the mean of the visible values), and for large scales whose wide score spread
+    # makes the running maximum grow by more than 2^8 often (rescaling the accumulated output);
+    # ragged chunks, decode rows, g = 4
+    ctx, nq = [300, 77, 513, 1], [129, 77, 1, 1]
+    case, q, q_start = _prefill_case(ctx, nq, 8, 2, 128, 16, dtype, 640)
+    ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens, scale,
+                             n_threads=0)
+    dev = case.to("cuda")
+    out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                         max_context_len=max(ctx), max_q_len=max(nq), scale=scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _assert_close(out.cpu(), ref, dtype, f"prefill {prefill_consumer} scale={scale}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("g", [1, 8])
+def test_prefill_mixed_batch_mma_sync(oracle_mod, monkeypatch, dtype, g):
+    monkeypatch.setenv("PA_PREFILL_CONSUMER", "mma_sync")
+    test_prefill_mixed_batch(oracle_mod, dtype, g, 128, 16)
+
+
+@pytest.mark.parametrize("scale", [-0.2, 0.0])
+def test_decode_scale_sign(oracle_mod, consumer, scale):
+    case = W.paged_case("dec-scale", [1, 17, 300, 1000], 8, 2, 128, 16, torch.bfloat16, 660)
+    ref = oracle_mod.decode(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens, scale)
+    dev = case.to("cuda")
+    out = api.pa_decode(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                        max_context_len=1000, scale=scale, out_dtype=torch.float32, partition_size=256)
+    torch.cuda.synchronize()
+    _assert_close(out.cpu(), ref, torch.bfloat16, f"decode {consumer} scale={scale}")
+
+
 def test_prefill_single_tokens_match_decode():
     case = W.gqa8k_bf16(S=32)
     dev = case.to("cuda")
