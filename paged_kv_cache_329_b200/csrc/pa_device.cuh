@@ -219,6 +219,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// Same, with A read from tensor memory: a_tmem addresses M lanes x (16 / 2) columns holding the
+// 16-bit A elements of one K = 16 slice packed in pairs (row m in lane m, element k in column k/2,
+// even k in the low half), which is what a 32x32b tcgen05.st of packed pairs leaves there.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -285,9 +297,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Split two fp32 values into a 16-bit pair hi and a 16-bit pair lo with x = hi + lo to about 16
+// Split two fp32 values into a 16-bit pair hi and a 16-bit pair lo with x = hi + lo to about 15
 // significant bits (element 0 in the low half of each word).  bf16: hi is x cut to its top 16 bits
-// (a byte permute), lo = x - hi is exact in fp32 and then rounded.  fp16: hi is rounded, lo likewise.
+// (a byte permute), lo = x - hi is exact in fp32 and is cut the same way (|error| < 2^-14 |x|, no
+// conversion instruction).  fp16: hi is rounded, lo = x - hi rounded.
 template <class T>
 struct Split;
 template <>
@@ -296,8 +309,7 @@ struct Split<__nv_bfloat16> {
     const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
     asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi) : "r"(b0), "r"(b1));
     const float l0 = x0 - __uint_as_float(b0 & 0xffff0000u), l1 = x1 - __uint_as_float(b1 & 0xffff0000u);
-    const __nv_bfloat162 v = __floats2bfloat162_rn(l0, l1);
-    lo = *reinterpret_cast<const uint32_t*>(&v);
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(lo) : "r"(__float_as_uint(l0)), "r"(__float_as_uint(l1)));
   }
 };
 template <>
@@ -310,6 +322,23 @@ struct Split<__half> {
     lo = *reinterpret_cast<const uint32_t*>(&l);
   }
 };
+
+// Store 32 consecutive 32-bit columns of this warp's 32 lanes; complete (visible to the tensor
+// core after a thread sync) once tmem_wait_st returns.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+      "%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32"
+      "};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -463,19 +463,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 // ---- tcgen05 consumers -------------------------------------------------------------------------------
 // 256 query rows per unit in two 128-row halves A and B (one TMEM lane per row in each half).
 // Warps 0-3 own the rows of half A, warps 4-7 those of half B (softmax, P, output); warp 8 is the
-// TMA producer; warp 9 allocates TMEM and one lane issues the MMAs.  Per 64-key tile j and half h:
+// TMA producer; one lane of warp 9 issues the MMAs of half A, one lane of warp 10 those of half B
+// (a single thread issues one tcgen05.mma about every 100 cycles whatever its size, so one issuer
+// per half doubles the rate at which these small MMAs reach the tensor core); warp 9 also
+// allocates TMEM.  Per 64-key tile j and half h:
 //   S_h[128 x 64]  = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
-//   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) to smem
-//   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    B = V tile (MN-major: d contiguous)
-// The MMA issue order S_A(j+1) before PV_B(j) lets one half's softmax run while the tensor core
-// serves the other half.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
+//   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) back to TMEM
+//   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    A = P_h from TMEM, B = V tile (MN-major: d contiguous)
+// The halves are independent pipelines that share the K/V ring, so one half's softmax runs while the
+// tensor core serves the other half.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
 // when a row's maximum grows by more than 2^8, which keeps every exponent bounded.
 constexpr int kURows = 128;                  // rows per half (TMEM lanes)
 constexpr int kUHalves = 2;
 constexpr int kUUnitRows = kURows * kUHalves;
-constexpr int kUProducer = 8, kUMma = 9;
-constexpr int kUThreads = 10 * 32;
-constexpr uint32_t kTmemCols = 512;          // S_A 0..63, S_B 64..127, O_A 128.., O_B 128+d..
+constexpr int kUProducer = 8, kUMma = 9;    // MMA issuers: warps kUMma (half A) and kUMma + 1 (half B)
+constexpr int kUThreads = 11 * 32;
+constexpr uint32_t kTmemCols = 512;          // S_A 0..63, S_B 64..127, O_A 128.., O_B 128+d.., P_A 384.., P_B 448..
+constexpr uint32_t kTmemP = 384;             // P_h: 32 columns of packed hi pairs, then 32 of lo pairs
 
 template <int D>
 struct UCfg {
@@ -483,20 +487,18 @@ struct UCfg {
   static constexpr int kPanelBytes = kTile * 128;
   static constexpr int kKVBytes = kNPanel * kPanelBytes;
   static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kStages = kNPanel == 1 ? 6 : 3;
+  static constexpr int kStages = kNPanel == 1 ? 8 : 5;
   static constexpr int kQPanelBytes = kURows * 128;
   static constexpr int kQHalfBytes = kNPanel * kQPanelBytes;
-  static constexpr int kPHalfBytes = 2 * kURows * 128;           // hi then lo: [128 rows][64 keys] each
   static constexpr int kOffQ = kStages * kStageBytes;
-  static constexpr int kOffP = kOffQ + kUHalves * kQHalfBytes;
-  static constexpr int kOffMeta = kOffP + kUHalves * kPHalfBytes;
+  static constexpr int kOffMeta = kOffQ + kUHalves * kQHalfBytes;
   static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
-  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done; then teardown
-  static constexpr int kNBars = 2 * kStages + 4 * kUHalves + 1;
+  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done, turn; then teardown
+  static constexpr int kNBars = 2 * kStages + 5 * kUHalves + 1;
   static constexpr int kOffTmem = kOffBar + kNBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(128 + kUHalves * D <= static_cast<int>(kTmemCols), "TMEM columns: two S tiles and two O tiles");
+  static_assert(128 + kUHalves * D <= static_cast<int>(kTmemP), "TMEM columns: two S tiles and two O tiles below P");
 };
 
 template <class T, int D, int G>
@@ -517,19 +519,21 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   uint64_t* s_full = q_ready + kUHalves;       // [2]
   uint64_t* p_full = s_full + kUHalves;        // [2]
   uint64_t* o_done = p_full + kUHalves;        // [2]
-  uint64_t* teardown = o_done + kUHalves;
+  uint64_t* turn = o_done + kUHalves;          // [2]: turn[h] = the other half finished a softmax
+  uint64_t* teardown = turn + kUHalves;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       pa::mbar_init(&full[i], 1);
-      pa::mbar_init(&empty[i], 1);  // one tcgen05.commit per tile
+      pa::mbar_init(&empty[i], kUHalves);  // one tcgen05.commit per tile from each half's issuer
     }
     for (int h = 0; h < kUHalves; ++h) {
       pa::mbar_init(&q_ready[h], kURows);
       pa::mbar_init(&s_full[h], 1);
       pa::mbar_init(&p_full[h], kURows);
       pa::mbar_init(&o_done[h], 1);
+      pa::mbar_init(&turn[h], kURows);
     }
     pa::mbar_init(teardown, kUUnitRows);
     pa::fence_barrier_init();
@@ -549,56 +553,48 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     return;
   }
 
-  if (warp == kUMma) {
-    // ================================ MMA issuer ==============================================
+  if (warp == kUMma || warp == kUMma + 1) {
+    // ================================ MMA issuers (one per half) ==============================
+    const int h = warp - kUMma;
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, q_ph = 0, p_ph[2] = {0, 0};
-      const uint32_t q_base = pa::smem_addr(smem + C::kOffQ);
-      const uint32_t p_base = pa::smem_addr(smem + C::kOffP);
+      uint32_t phase = 0, q_ph = 0, p_ph = 0;
+      const uint32_t q_base = pa::smem_addr(smem + C::kOffQ) + h * C::kQHalfBytes;
       bool ok = true;
-      // A half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
-      // MMAs, but its barriers are committed all the same so that both sides count the same phases.
-      auto issue_s = [&](int h, int st, bool active) {
-        if (active) {
-          const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
-          const uint32_t qb = q_base + h * C::kQHalfBytes;
-#pragma unroll
-          for (int k = 0; k < KS; ++k) {
-            const uint64_t da = pa::sw128_desc(qb + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
-            const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-            pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
-          }
-        }
-        pa::umma_commit(&s_full[h]);
+      // One K = 16 step of S_h = Q_h K^T (k over d) and one K = 16 step of O_h += P_h V (i over the
+      // hi keys, then the lo keys).
+      auto s_step = [&](int st, int k) {
+        const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
+        const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
+        const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
+        pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
       };
-      auto issue_pv = [&](int h, int st, bool first_tile, bool active) {
-        if (active) {
-          const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
-          const uint32_t pb = p_base + h * C::kPHalfBytes;
-#pragma unroll
-          for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              const uint64_t da = pa::sw128_desc(pb + part * (kURows * 128) + kk * 32, 16, 1024);
-              const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
-              const bool init = first_tile && part == 0 && kk == 0;
-              pa::umma_f16(tmem + 128 + D * h, da, db, kIdescO, init ? 0u : 1u);
-            }
-        }
-        pa::umma_commit(&o_done[h]);
+      auto pv_step = [&](int st, bool first_tile, int i) {
+        const int part = i / (kTile / 16), kk = i % (kTile / 16);
+        const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
+        const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
+        const bool init = first_tile && i == 0;
+        pa::umma_f16_tmem_a(tmem + 128 + D * h, tmem + kTmemP + 64 * h + part * 32 + kk * 8, db, kIdescO,
+                            init ? 0u : 1u);
       };
+      constexpr int kPV = 2 * (kTile / 16);
+      constexpr int kSteps = kPV > KS ? kPV : KS;
       while (ok) {
-        // first tile of a unit
+        // first tile of a unit: S_h(0)
         if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
         Meta mt = meta[stage];
         if (mt.flags & kDone) break;
-        if (!pa::mbar_wait(&q_ready[0], q_ph) || !pa::mbar_wait(&q_ready[1], q_ph)) { ok = false; break; }
+        if (!pa::mbar_wait(&q_ready[h], q_ph)) { ok = false; break; }
         q_ph ^= 1;
         pa::tc_fence_after();
-        const bool act_b = mt.nq * G > kURows;  // half A always holds the unit's first query
-        issue_s(0, stage, true);
-        issue_s(1, stage, act_b);
+        // a half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
+        // MMAs, but its barriers are committed all the same so that both sides count the same phases
+        const bool active = h == 0 || mt.nq * G > kURows;
+        if (active) {
+#pragma unroll
+          for (int k = 0; k < KS; ++k) s_step(stage, k);
+        }
+        pa::umma_commit(&s_full[h]);
         bool first = true;
         while (true) {
           const bool last = (mt.flags & kLast) != 0;
@@ -608,21 +604,22 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
             nstage = 0;
             nphase ^= 1;
           }
-          if (!pa::mbar_wait(&p_full[0], p_ph[0])) { ok = false; break; }
-          p_ph[0] ^= 1;
+          if (!last && !pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
+          if (!pa::mbar_wait(&p_full[h], p_ph)) { ok = false; break; }
+          p_ph ^= 1;
           pa::tc_fence_after();
-          issue_pv(0, stage, first, true);
-          if (!last) {
-            if (!pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
-            pa::tc_fence_after();
-            issue_s(0, nstage, true);
+          // O_h += P_h(j) V_j and, when there is a next tile, S_h(j+1) = Q_h K_{j+1}^T, alternating
+          // step by step (independent accumulators)
+          if (active) {
+#pragma unroll
+            for (int i = 0; i < kSteps; ++i) {
+              if (i < kPV) pv_step(stage, first, i);
+              if (!last && i < KS) s_step(nstage, i);
+            }
           }
-          if (!pa::mbar_wait(&p_full[1], p_ph[1])) { ok = false; break; }
-          p_ph[1] ^= 1;
-          pa::tc_fence_after();
-          issue_pv(1, stage, first, act_b);
+          pa::umma_commit(&o_done[h]);
+          if (!last) pa::umma_commit(&s_full[h]);
           pa::umma_commit(&empty[stage]);
-          if (!last) issue_s(1, nstage, act_b);
           stage = nstage;
           phase = nphase;
           if (last) break;
@@ -632,6 +629,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       }
       if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
     }
+    if (h == 1) return;
     __syncwarp();
     // free TMEM once the row threads are done with it
     pa::mbar_wait(teardown, 0);
@@ -646,16 +644,15 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   const int r = half * kURows + hr;                   // row within the unit
   const int warp_row0 = half * kURows + (warp & 3) * 32;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tS = tmem + 64 * half, tO = tmem + 128 + D * half;
+  const uint32_t tS = tmem + 64 * half, tO = tmem + 128 + D * half, tP = tmem + kTmemP + 64 * half;
   uint8_t* qs = smem + C::kOffQ + half * C::kQHalfBytes;
-  uint8_t* ph = smem + C::kOffP + half * C::kPHalfBytes;
-  uint8_t* pl = ph + kURows * 128;
   uint64_t* my_q_ready = &q_ready[half];
   uint64_t* my_s_full = &s_full[half];
   uint64_t* my_p_full = &p_full[half];
   uint64_t* my_o_done = &o_done[half];
   int stage = 0;
-  uint32_t phase = 0, s_ph = 0, o_ph = 0;
+  uint32_t phase = 0, s_ph = 0, o_ph = 0, t_ph = 0;
+  bool first_turn = half == 0;                        // half A takes the first softmax
   float m_used = -INFINITY, l = 0.f;
   int row_global = -1, qpos = 0;
   bool pv_pending = false, ok = true, warp_active = false;
@@ -692,17 +689,26 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       l = 0.f;
     }
     // keys past the tile's valid ones get p = 0; zero their V rows, which may hold stale or unused
-    // data (half A does it: both halves' P.V products are issued after half A's P is ready)
-    if (mt.ntok < kTile && half == 0) {
+    // data.  Each half does it before its own P.V product is issued (the two write the same zeros),
+    // and makes the writes visible to the tensor core.
+    if (mt.ntok < kTile) {
       uint8_t* vs = smem + stage * C::kStageBytes + C::kKVBytes;
       for (int i = hr; i < (kTile - mt.ntok) * (D / 8); i += kURows) {
         const int row = mt.ntok + i / (D / 8), c = i % (D / 8);
         *reinterpret_cast<uint4*>(vs + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
             make_uint4(0u, 0u, 0u, 0u);
       }
+      pa::fence_proxy_async_smem();
     }
     if (!pa::mbar_wait(my_s_full, s_ph)) { ok = false; break; }
     s_ph ^= 1;
+    // the halves take turns at the softmax, so that each has the SFUs to itself while the tensor
+    // core works for the other
+    if (!first_turn) {
+      if (!pa::mbar_wait(&turn[half], t_ph)) { ok = false; break; }
+      t_ph ^= 1;
+    }
+    first_turn = false;
     // S(j) is issued after this half's P.V(j-1), so that product is complete as well
     if (pv_pending) {
       if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
@@ -751,25 +757,22 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       // p = 2^(s * sl2 - m); with no visible key so far every s is -inf and p = 0
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t hi[kTile / 2], lo[kTile / 2];
 #pragma unroll
-      for (int c8 = 0; c8 < kTile / 8; ++c8) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = pa::ex2(fmaf(sv[8 * c8 + 2 * e], sl2, neg_m));
-          const float p1 = pa::ex2(fmaf(sv[8 * c8 + 2 * e + 1], sl2, neg_m));
-          ls[e] += p0 + p1;
-          pa::Split<T>::run(p0, p1, hi[e], lo[e]);
-        }
-        const int off = hr * 128 + ((c8 ^ (hr & 7)) << 4);
-        *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      for (int k2 = 0; k2 < kTile / 2; ++k2) {
+        const float p0 = pa::ex2(fmaf(sv[2 * k2], sl2, neg_m));
+        const float p1 = pa::ex2(fmaf(sv[2 * k2 + 1], sl2, neg_m));
+        ls[k2 & 3] += p0 + p1;
+        pa::Split<T>::run(p0, p1, hi[k2], lo[k2]);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      pa::fence_proxy_async_smem();
+      pa::tmem_st32(tP + lane_base, hi);
+      pa::tmem_st32(tP + lane_base + 32, lo);
+      pa::tmem_wait_st();
     }
     pa::tc_fence_before();
     pa::mbar_arrive(my_p_full);
+    pa::mbar_arrive(&turn[half ^ 1]);
     pv_pending = true;
     if (mt.flags & kLast) {
       if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
