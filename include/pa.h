@@ -295,6 +295,22 @@ pa_status pa_step_run(pa_step* step, void* stream);
  * next step's inputs on the host while the GPU runs the current one. */
 pa_status pa_step_launch(pa_step* step, void* stream);
 
+/* Pipelined form of pa_step_launch: returns at once, and the step's transfers overlap the kernels
+ * of neighbouring steps.  The host->device copy of the inputs runs on a copy stream of the step
+ * (after this step's previous kernels are done with its device inputs); the kernels (copy-on-write
+ * copy, cache write, decode; captured once as a graph) run on `stream` once that copy has landed
+ * and this step's previous output copy has left d_out; the device->host copy of the output runs on
+ * a second copy stream once the kernels are done.  All kernels of all steps launched on one
+ * `stream` run in launch order, so the caches see the steps in order.  The caller may refill this
+ * step's host inputs, and read h_out, only after pa_step_wait(step).  With two steps (two sets of
+ * buffers) launched alternately, step i+1's input copy and step i-1's output copy overlap step i's
+ * kernels. */
+pa_status pa_step_launch_async(pa_step* step, void* stream);
+
+/* Blocks until the output copy of this step's last pa_step_launch_async has completed (at once if
+ * there was none). */
+pa_status pa_step_wait(pa_step* step);
+
 void pa_step_destroy(pa_step* step);
 
 /* ---------------------------------------------------------------------------------------------

@@ -51,6 +51,8 @@ SIGNATURES = {
     "pa_step_create": (P, [ctypes.POINTER(StepDesc)]),
     "pa_step_run": (I, [P, P]),
     "pa_step_launch": (I, [P, P]),
+    "pa_step_launch_async": (I, [P, P]),
+    "pa_step_wait": (I, [P]),
     "pa_step_destroy": (None, [P]),
     "pa_alloc_create": (P, [I, I]),
     "pa_alloc_destroy": (None, [P]),

@@ -241,6 +241,17 @@ class DecodeStep:
         """Enqueue the step and return; h_out is valid once the stream reaches it."""
         _check(self._lib.pa_step_launch(self._h, _stream(stream)))
 
+    def launch_async(self, stream=None):
+        """Enqueue the step with its input and output copies on the step's own copy streams, so
+        that they overlap neighbouring steps' kernels.  Refill the host inputs and read h_out only
+        after wait()."""
+        _check(self._lib.pa_step_launch_async(self._h, _stream(stream)))
+
+    def wait(self):
+        """Block until the output of the last launch_async() is in h_out."""
+        _check(self._lib.pa_step_wait(self._h))
+        return self.h_out
+
     def __del__(self):
         h = getattr(self, "_h", None)
         if h:

@@ -314,6 +314,58 @@ def test_captured_step_matches_separate_calls(oracle_mod):
     assert api.workspace_error(step.workspace) == 0
 
 
+def test_pipelined_steps_match_oracle(oracle_mod):
+    # Two captured steps launched alternately with launch_async: step i+1's input copy and step
+    # i-1's output copy overlap step i's kernels.  Every output must equal the oracle applied to the
+    # block manager state of its own step, and the caches must end bit-identical.
+    B, H, Hk, d, dt = 16, 32, 8, 128, torch.bfloat16
+    mgr = api.BlockManager(512, B)
+    g = W.generator(410)
+    kc = W.randn(g, (512, Hk, B, d), dt)
+    vc = W.randn(g, (512, Hk, B, d), dt)
+    roots = []
+    for r in range(4):
+        root = mgr.seq_create()
+        mgr.reserve_slots(root, 150 + 29 * r)
+        roots.append([root] + [mgr.seq_fork(root) for _ in range(3)])
+    kd, vd = kc.cuda(), vc.cuda()
+    S = 16
+    steps = [api.DecodeStep(kd, vd, S, H, 32, 512, out_dtype=torch.float32) for _ in range(2)]
+    k_ref, v_ref = kc.clone(), vc.clone()
+    rnd = torch.Generator().manual_seed(11)
+    stream = torch.cuda.current_stream()
+    refs = {}
+    n_steps = 7
+    for it in range(n_steps):
+        step = steps[it % 2]
+        if it >= 2:
+            _assert_close(step.wait().clone(), refs.pop(it - 2), dt, f"pipelined step {it - 2}")
+        seqs = []
+        for gi, beams in enumerate(roots):
+            parents = torch.randint(0, 4, (4,), generator=rnd).tolist()
+            kids = [mgr.seq_fork(beams[p]) for p in parents]
+            for b in beams:
+                mgr.seq_free(b)
+            roots[gi] = kids
+            seqs += kids
+        slots, pairs = mgr.reserve_slots_batch(seqs, 1, step.h_slots)
+        mgr.build_block_tables(seqs, 32, step.h_tables, step.h_lens)
+        step.set_pairs(pairs)
+        step.h_query.copy_(W.randn(g, (S, H, d), dt))
+        step.h_key.copy_(W.randn(g, (S, Hk, d), dt))
+        step.h_value.copy_(W.randn(g, (S, Hk, d), dt))
+        step.launch_async(stream)
+        k_ref, v_ref = oracle_mod.copy_blocks(k_ref, v_ref, pairs)
+        k_ref, v_ref = oracle_mod.cache_write(k_ref, v_ref, step.h_key, step.h_value, step.h_slots)
+        refs[it] = oracle_mod.decode(step.h_query, k_ref, v_ref, step.h_tables, step.h_lens)
+    for it in (n_steps - 2, n_steps - 1):
+        _assert_close(steps[it % 2].wait().clone(), refs.pop(it), dt, f"pipelined step {it}")
+    torch.cuda.synchronize()
+    assert torch.equal(kd.cpu().view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(vd.cpu().view(torch.int16), v_ref.view(torch.int16))
+    assert all(api.workspace_error(st.workspace) == 0 for st in steps)
+
+
 # ---- swap to pinned host memory and back (pa_swap_blocks) --------------------------------------------
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
