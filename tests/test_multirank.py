@@ -61,3 +61,38 @@ def test_reference_arm_under_torchrun_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _dying_worker(rank, world, port, q):
+    import datetime
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    sys.path.insert(0, ROOT)
+    import bench
+
+    if rank == 1:
+        raise SystemExit(3)                        # leaves between steps, before the timing collective
+    t0 = time.time()
+    try:
+        bench.reduce_max([1.0], world)
+        q.put(("returned", time.time() - t0))
+    except Exception as e:                         # the survivor learns of it from the collective
+        q.put(("error", time.time() - t0, type(e).__name__))
+
+
+def test_rank_that_leaves_ends_the_collective_with_an_error():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_dying_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert res[0] == "error", res                 # no hang, no silent result
+    assert res[1] < 60.0
+    assert procs[1].exitcode == 3
