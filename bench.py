@@ -41,6 +41,7 @@ from paged_kv_cache_329_b200 import api  # noqa: E402
 from paged_kv_cache_329_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode-attn effective KV GB/s (% of B200 HBM peak); seqs/s per step"
+L2_BYTES = 126e6   # B200 L2
 
 
 # ---- workload -----------------------------------------------------------------------------------
@@ -57,6 +58,9 @@ WORKLOADS = {
                                     "a 1024-token prompt (64 blocks at ref count 4), tails U[0,256]; every step "
                                     "each sequence forks from a seeded parent among its request's 4, so shared "
                                     "partial tail blocks are copied on write"),
+    "tiny_fp32": dict(S=4, H=8, Hk=8, d=64, B=16, dtype=torch.float32,
+                      lens=lambda: W.lens_uniform(W.generator(1), 4, 1, 200),
+                      desc="tiny fp32 paged decode: 4 seqs, 8 q heads = 8 kv heads, d=64, B=16, context U[1,200]"),
     "long_bf16": dict(S=16, H=64, Hk=8, d=128, B=16, dtype=torch.bfloat16,
                       lens=lambda: W.lens_uniform(W.generator(5), 16, 16384, 32768),
                       desc="long-context bf16: 16 seqs, 64 q / 8 kv heads, d=128, B=16, context U[16384,32768]"),
@@ -66,8 +70,11 @@ WORKLOADS = {
 class Workload:
     """Sequences in a native block manager over a shuffled pool, random K/V in HBM."""
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0):
-        cfg = WORKLOADS[name]
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
+        cfg = dict(WORKLOADS[name])
+        if block_size:
+            cfg["B"] = block_size
+            cfg["desc"] = cfg["desc"].replace("B=16", f"B={block_size}")
         self.name, self.cfg = name, cfg
         self.S, self.H, self.Hk, self.d, self.B, self.dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
         self.es = torch.finfo(self.dtype).bits // 8
@@ -136,9 +143,9 @@ class SharedPrefixWorkload(Workload):
 
     REQUESTS, WIDTH, PROMPT, TAIL_MAX = 32, 4, 1024, 256
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0):
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
         self.rnd = torch.Generator().manual_seed(4 + seed_offset)
-        super().__init__(name, device, seed_offset, growth_steps + 64, partition)
+        super().__init__(name, device, seed_offset, growth_steps + 64, partition, block_size)
 
     def _lengths(self):
         tails = torch.randint(0, self.TAIL_MAX + 1, (self.REQUESTS * self.WIDTH,), generator=self.rnd)
@@ -182,9 +189,9 @@ class SharedPrefixWorkload(Workload):
         return len(used) * self.Hk * self.B * self.d * 2 * self.es
 
 
-def make_workload(name, device, seed_offset=0, growth_steps=0, partition=0):
+def make_workload(name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
     cls = SharedPrefixWorkload if name == "shared_prefix_bf16" else Workload
-    return cls(name, device, seed_offset, growth_steps, partition)
+    return cls(name, device, seed_offset, growth_steps, partition, block_size)
 
 
 def load_peaks():
@@ -286,7 +293,7 @@ def run_pa(args, rank, world, local_rank):
     e2e_steps = min(K, args.e2e_steps)
     n_traj = 32 if args.workload == "shared_prefix_bf16" else 1
     wl = make_workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + n_traj + 2,
-                       partition=args.partition)
+                       partition=args.partition, block_size=args.block_size)
     S, H, Hk, d = wl.S, wl.H, wl.Hk, wl.d
     gen = torch.Generator(device=dev).manual_seed(99 + rank)
     q = torch.randn((S, H, d), generator=gen, device=dev).to(wl.dtype)
@@ -430,7 +437,9 @@ def run_pa(args, rank, world, local_rank):
             "seq_len": f"mean {statistics.mean(lens.tolist()):.0f}, max {max(lens.tolist())}",
             "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
             "partition_size": wl.P,
-            "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush",
+            "l2": (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush"
+                   if kv_bytes > L2_BYTES else
+                   f"warm: the {kv_bytes / 1e6:.1f} MB of K/V read per step fit in L2 (no flush)"),
             "step": "host block manager -> pa_copy_blocks -> pa_cache_write -> pa_decode (plan, decode, combine)",
             "step_bytes": round(step_bytes),
             "cow_pairs_per_step": n_pairs,
@@ -728,8 +737,10 @@ def run_reference(args, rank, world):
     import oracle
 
     oracle.build()
-    cfg = WORKLOADS[args.workload]
-    lens = cfg["lens"]().tolist()
+    cfg = dict(WORKLOADS[args.workload])
+    if args.block_size:
+        cfg["B"] = args.block_size
+    lens = cfg["lens"]().tolist() if cfg["lens"] else [1024 + 128] * cfg["S"]   # shared prefix: prompt + mean tail
     S, H, Hk, d, B, dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
     es = torch.finfo(dtype).bits // 8
     cores = oracle.hardware_threads()
@@ -797,6 +808,7 @@ def main():
     ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS) + ["swap_bf16", "prefill_mixed_bf16", "cache_ops_bf16"])
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--partition", type=int, default=0, help="decode partition size in tokens (0 = library default)")
+    ap.add_argument("--block-size", type=int, default=0, help="tokens per KV block (0 = the workload's own)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
