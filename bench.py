@@ -42,6 +42,7 @@ from paged_kv_cache_329_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode-attn effective KV GB/s (% of B200 HBM peak); seqs/s per step"
 L2_BYTES = 126e6   # B200 L2
+E2E_DEPTH = 3      # decode steps in flight in the end-to-end leg
 
 
 # ---- workload -----------------------------------------------------------------------------------
@@ -203,8 +204,11 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if its source hash matches."""
+def profiled_traffic(args):
+    """DRAM bytes per decode launch from the committed ncu summary, if its source hash matches and
+    the run is the workload it was captured on (gqa8k_bf16, library-default partition and B)."""
+    if args.workload != "gqa8k_bf16" or args.partition or args.block_size:
+        return None
     path = os.path.join(ROOT, "profiles", "decode_kernel_gqa8k_bf16.md")
     src = os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", "pa_decode.cu")
     try:
@@ -218,21 +222,44 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed loops run."""
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loops run.  A reader
+    thread collects the samples; the constructor returns once sampling has started, and a timed
+    window shorter than the sampling interval takes the samples nearest to it."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
-        self.proc = None
-        self.windows = []
+        import threading
+
+        self.proc, self.windows, self.samples = None, [], []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.02)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                whole, _, frac = f[0].partition(".")
+                ts = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + (float("0." + frac) if frac else 0.0)
+                sm, mx = float(f[1]), float(f[2])
+            except Exception:
+                continue
+            self.samples.append((ts, sm, mx, [n for n, v in zip(self.NAMES, f[4:8]) if v.lower() == "active"]))
 
     def mark(self, t0, t1):
         self.windows.append((t0, t1))
@@ -243,32 +270,21 @@ class ClockSampler:
         time.sleep(0.1)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            return None
-        sms, maxes, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
-                sm, mx = float(f[1]), float(f[2])
-            except Exception:
-                continue
-            if not any(a - 1.0 <= ts <= b + 1.0 for a, b in self.windows):
-                continue
-            sms.append(sm)
-            maxes.append(mx)
-            for n, v in zip(names, f[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sms:
+        self.thread.join(timeout=5)
+        picked = []
+        for a, b in self.windows:
+            inside = [x for x in self.samples if a <= x[0] <= b]
+            if not inside and self.samples:     # window shorter than the sampling interval
+                inside = sorted(self.samples, key=lambda x: min(abs(x[0] - a), abs(x[0] - b)))[:2]
+            picked += inside
+        if not picked:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
-                "samples": len(sms)}
+        reasons = sorted({n for x in picked for n in x[3]})
+        return {"sm_mhz": statistics.median(x[1] for x in picked), "sm_max_mhz": max(x[2] for x in picked),
+                "reasons": reasons, "samples": len(picked)}
 
 
 def reduce_max(values, world, device="cpu"):
@@ -360,12 +376,12 @@ def run_pa(args, rank, world, local_rank):
     launches_total = sum(launches[i % n_traj] for i in range(K))
 
     # ---- end to end through the API: captured steps replayed from pinned host memory ----
-    # Two captured steps (two sets of buffers) launched alternately with launch_async: the host
-    # block manager prepares step i while the GPU runs step i-1; step i's input copy and step
-    # i-1's output copy run on copy streams beside step i-1's and step i's kernels.  A step's
-    # buffers are refilled only after its previous output has come back (wait()).
+    # E2E_DEPTH captured steps (sets of buffers) launched in turn with launch_async: the host block
+    # manager prepares step i while the GPU runs the steps before it; step i's input copy and the
+    # previous steps' output copies run on copy streams beside the kernels.  A step's buffers are
+    # refilled only after its previous output has come back (wait()).
     steps = [api.DecodeStep(wl.k_cache, wl.v_cache, S, H, wl.max_blocks, wl.max_c, max_pairs=S,
-                            out_dtype=wl.dtype, partition_size=wl.P) for _ in range(2)]
+                            out_dtype=wl.dtype, partition_size=wl.P) for _ in range(E2E_DEPTH)]
     for st in steps:
         st.h_query.copy_(q.cpu())
         st.h_key.copy_(key.cpu())
@@ -384,12 +400,12 @@ def run_pa(args, rank, world, local_rank):
 
     def e2e_run(n):
         for i in range(n):
-            st = steps[i % 2]
-            if i >= 2:
-                st.wait()                # step i-2's output is in st.h_out; its buffers are free
-            prepare(st)                  # overlaps the GPU running step i-1
+            st = steps[i % E2E_DEPTH]
+            if i >= E2E_DEPTH:
+                st.wait()                # step i-E2E_DEPTH's output is in st.h_out; its buffers are free
+            prepare(st)                  # overlaps the GPU running the previous steps
             st.launch_async(stream)
-        for st in steps[:min(n, 2)]:
+        for st in steps[:min(n, E2E_DEPTH)]:
             st.wait()
         stream.synchronize()
 
@@ -461,7 +477,7 @@ def run_pa(args, rank, world, local_rank):
             "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic(),
+            "traffic": profiled_traffic(args),
             "algorithmic_bytes_per_launch": decode_bytes,
             "launch_ms": round(decode_ms, 5),
         },
@@ -476,8 +492,8 @@ def run_pa(args, rank, world, local_rank):
             "note": "per step: host block manager (prepared while the GPU runs the previous step), H2D "
                     "of the step's inputs from pinned memory, one replay of the captured kernels "
                     "(copy_blocks, cache_write, decode), D2H of o; the copies run on copy streams beside the "
-                    "neighbouring steps' kernels; every step's output is read back (at most two steps "
-                    "in flight)",
+                    "neighbouring steps' kernels; every step's output is read back (at most "
+                    f"{E2E_DEPTH} steps in flight)",
         },
         "gpu_launches": launches_total,
     }
