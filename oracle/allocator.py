@@ -17,7 +17,7 @@ Rules followed (page title, section):
   * "Paged Attention&Orca Paper笔记与解读", parallel sampling and beam search: sequences fork by
     sharing blocks; a block whose count drops to 0 is freed.
 
-Readings where the pages are open (each listed in the design doc):
+Readings where the pages are open:
   * The last block full: the next token gets a fresh block with no copy, even if the full block is
     shared.  Partial and shared: copy-on-write.  Partial and count 1: in place.
   * Free-block policy: a LIFO stack that starts as [n-1, ..., 1, 0], so the first allocation

@@ -13,7 +13,7 @@
 //   [P2-COW]   "PagedAttention原理", section "解决COW", five-step copy-on-write list
 //   [P4-DEC]   "vllm" (cnblogs), section 2.2 Decode: each decode step stores the new token's K,V
 //
-// Readings taken where the pages leave a step open (all listed in the design doc):
+// Readings taken where the pages leave a step open:
 //   * query head h reads kv head h / g with g = H / Hk (grouped-query attention, contiguous groups);
 //   * the last block of a sequence holds c - (nb-1)*B valid tokens; only t < c contributes;
 //   * the score scale is passed in (1/sqrt(d) by default);
