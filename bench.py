@@ -669,11 +669,14 @@ def run_prefill(args, rank, world, local_rank):
     if rank != 0:
         return None
     tflops = world * flops * args.steps / (ms * 1e-3) / 1e12
+    # the launches run back to back for about a second under the power cap: the sustained figure
+    # is the denominator, the burst one is reported beside it
     try:
-        peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
-        kind = "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak, burst = float(peaks["bf16_tflops_sustained"]), float(peaks["bf16_tflops"])
+        kind = "measured (MEASURED_PEAKS.json bf16_tflops_sustained, cuBLAS back to back for 4 s)"
     except Exception:
-        peak, kind = 1590.0, "fallback"
+        peak, burst, kind = 1400.0, 1590.0, "fallback (sustained)"
     return {"metric": "paged prefill + decode attention TFLOP/s (mixed batch)", "value": round(tflops, 2),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
@@ -683,7 +686,8 @@ def run_prefill(args, rank, world, local_rank):
                        "flops_per_step": flops, "unique_kv_bytes": kv_bytes},
             "kv_gbs_unique": round(world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, 2),
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak, "peak_kind": kind,
-                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4), "traffic": None},
+                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4), "traffic": None,
+                         "peak_burst": burst, "frac_of_burst": round(tflops / world / burst, 4)},
             "clocks": clock_info, "gpu_launches": 2 * args.steps}
 
 

@@ -470,8 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 //   S_h[128 x 64]  = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
 //   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) back to TMEM
 //   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    A = P_h from TMEM, B = V tile (MN-major: d contiguous)
-// The halves are independent pipelines that share the K/V ring, so one half's softmax runs while the
-// tensor core serves the other half.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
+// The halves are independent pipelines that share the K/V ring.  S_h(j+1) is issued as soon as the
+// rows have read S_h(j) out of TMEM, so it runs during their softmax of tile j and only P.V(j) waits
+// for P.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
 // when a row's maximum grows by more than 2^8, which keeps every exponent bounded.
 constexpr int kURows = 128;                  // rows per half (TMEM lanes)
 constexpr int kUHalves = 2;
@@ -493,7 +494,7 @@ struct UCfg {
   static constexpr int kOffQ = kStages * kStageBytes;
   static constexpr int kOffMeta = kOffQ + kUHalves * kQHalfBytes;
   static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
-  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done, turn; then teardown
+  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done, s_free; then teardown
   static constexpr int kNBars = 2 * kStages + 5 * kUHalves + 1;
   static constexpr int kOffTmem = kOffBar + kNBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;
@@ -519,8 +520,8 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   uint64_t* s_full = q_ready + kUHalves;       // [2]
   uint64_t* p_full = s_full + kUHalves;        // [2]
   uint64_t* o_done = p_full + kUHalves;        // [2]
-  uint64_t* turn = o_done + kUHalves;          // [2]: turn[h] = the other half finished a softmax
-  uint64_t* teardown = turn + kUHalves;
+  uint64_t* s_free = o_done + kUHalves;        // [2]: the rows of h have read S_h out of TMEM
+  uint64_t* teardown = s_free + kUHalves;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       pa::mbar_init(&s_full[h], 1);
       pa::mbar_init(&p_full[h], kURows);
       pa::mbar_init(&o_done[h], 1);
-      pa::mbar_init(&turn[h], kURows);
+      pa::mbar_init(&s_free[h], kURows);
     }
     pa::mbar_init(teardown, kUUnitRows);
     pa::fence_barrier_init();
@@ -558,7 +559,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     const int h = warp - kUMma;
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, q_ph = 0, p_ph = 0;
+      uint32_t phase = 0, q_ph = 0, p_ph = 0, f_ph = 0;
       const uint32_t q_base = pa::smem_addr(smem + C::kOffQ) + h * C::kQHalfBytes;
       bool ok = true;
       // One K = 16 step of S_h = Q_h K^T (k over d) and one K = 16 step of O_h += P_h V (i over the
@@ -578,7 +579,6 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
                             init ? 0u : 1u);
       };
       constexpr int kPV = 2 * (kTile / 16);
-      constexpr int kSteps = kPV > KS ? kPV : KS;
       while (ok) {
         // first tile of a unit: S_h(0)
         if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
@@ -604,21 +604,27 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
             nstage = 0;
             nphase ^= 1;
           }
-          if (!last && !pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
+          // S_h(j+1) as soon as the rows have read S_h(j) out of TMEM: it then runs during their
+          // softmax of tile j, and only P.V(j) waits for P
+          if (!pa::mbar_wait(&s_free[h], f_ph)) { ok = false; break; }
+          f_ph ^= 1;
+          if (!last) {
+            if (!pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
+            pa::tc_fence_after();
+            if (active) {
+#pragma unroll
+              for (int k = 0; k < KS; ++k) s_step(nstage, k);
+            }
+            pa::umma_commit(&s_full[h]);
+          }
           if (!pa::mbar_wait(&p_full[h], p_ph)) { ok = false; break; }
           p_ph ^= 1;
           pa::tc_fence_after();
-          // O_h += P_h(j) V_j and, when there is a next tile, S_h(j+1) = Q_h K_{j+1}^T, alternating
-          // step by step (independent accumulators)
           if (active) {
 #pragma unroll
-            for (int i = 0; i < kSteps; ++i) {
-              if (i < kPV) pv_step(stage, first, i);
-              if (!last && i < KS) s_step(nstage, i);
-            }
+            for (int i = 0; i < kPV; ++i) pv_step(stage, first, i);
           }
           pa::umma_commit(&o_done[h]);
-          if (!last) pa::umma_commit(&s_full[h]);
           pa::umma_commit(&empty[stage]);
           stage = nstage;
           phase = nphase;
@@ -651,8 +657,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   uint64_t* my_p_full = &p_full[half];
   uint64_t* my_o_done = &o_done[half];
   int stage = 0;
-  uint32_t phase = 0, s_ph = 0, o_ph = 0, t_ph = 0;
-  bool first_turn = half == 0;                        // half A takes the first softmax
+  uint32_t phase = 0, s_ph = 0, o_ph = 0;
   float m_used = -INFINITY, l = 0.f;
   int row_global = -1, qpos = 0;
   bool pv_pending = false, ok = true, warp_active = false;
@@ -702,23 +707,16 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     }
     if (!pa::mbar_wait(my_s_full, s_ph)) { ok = false; break; }
     s_ph ^= 1;
-    // the halves take turns at the softmax, so that each has the SFUs to itself while the tensor
-    // core works for the other
-    if (!first_turn) {
-      if (!pa::mbar_wait(&turn[half], t_ph)) { ok = false; break; }
-      t_ph ^= 1;
-    }
-    first_turn = false;
-    // S(j) is issued after this half's P.V(j-1), so that product is complete as well
-    if (pv_pending) {
-      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
-      o_ph ^= 1;
-      pv_pending = false;
-    }
     pa::tc_fence_after();
+    float sv[kTile];
+    if (warp_active) pa::tmem_ld64(tS + lane_base, sv);
+    // S_h may be overwritten by the next tile's S from here on
+    pa::tc_fence_before();
+    pa::mbar_arrive(&s_free[half]);
+    uint32_t hi[kTile / 2], lo[kTile / 2];
+    float f = 1.f;
+    bool rescale = false;
     if (warp_active) {
-      float sv[kTile];
-      pa::tmem_ld64(tS + lane_base, sv);
       // causal and length masking only on tiles that reach past the unit's first query position
       // or past the context (the same decision for the whole unit)
       if (mt.ntok < kTile || mt.tile_pos + kTile - 1 > mt.qpos0) {
@@ -733,31 +731,17 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
-      // tcgen05.ld/st are warp-collective, so the rescale of O is decided per warp; rows that do not
-      // need it take the factor 1
-      const bool grow = mx > m_used + 8.f;
-      if (__any_sync(0xffffffffu, grow)) {
-        float f = 1.f;
-        if (grow) {
-          if (m_used != -INFINITY) f = pa::ex2(m_used - mx);
-          l *= f;
-          m_used = mx;
-        }
-        if (!(mt.flags & kFirst) && __any_sync(0xffffffffu, f != 1.f)) {
-#pragma unroll 1
-          for (int j = 0; j < D / 16; ++j) {
-            float t[16];
-            pa::tmem_ld16(tO + lane_base + 16 * j, t);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) t[e] *= f;
-            pa::tmem_st16(tO + lane_base + 16 * j, t);
-          }
-        }
+      // the running maximum moves only when it grows by more than 2^8; O is then rescaled by f
+      // (below, once P.V(j-1) is done), decided per warp because tcgen05.ld/st are warp-collective
+      if (mx > m_used + 8.f) {
+        if (m_used != -INFINITY) f = pa::ex2(m_used - mx);
+        l *= f;
+        m_used = mx;
       }
+      rescale = !(mt.flags & kFirst) && __any_sync(0xffffffffu, f != 1.f);
       // p = 2^(s * sl2 - m); with no visible key so far every s is -inf and p = 0
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t hi[kTile / 2], lo[kTile / 2];
 #pragma unroll
       for (int k2 = 0; k2 < kTile / 2; ++k2) {
         const float p0 = pa::ex2(fmaf(sv[2 * k2], sl2, neg_m));
@@ -766,13 +750,31 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
         pa::Split<T>::run(p0, p1, hi[k2], lo[k2]);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+    }
+    // P.V(j-1) must be complete before P is rewritten and O rescaled
+    if (pv_pending) {
+      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
+      o_ph ^= 1;
+      pv_pending = false;
+    }
+    pa::tc_fence_after();
+    if (warp_active) {
+      if (rescale) {
+#pragma unroll 1
+        for (int j = 0; j < D / 16; ++j) {
+          float t[16];
+          pa::tmem_ld16(tO + lane_base + 16 * j, t);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t[e] *= f;
+          pa::tmem_st16(tO + lane_base + 16 * j, t);
+        }
+      }
       pa::tmem_st32(tP + lane_base, hi);
       pa::tmem_st32(tP + lane_base + 32, lo);
       pa::tmem_wait_st();
     }
     pa::tc_fence_before();
     pa::mbar_arrive(my_p_full);
-    pa::mbar_arrive(&turn[half ^ 1]);
     pv_pending = true;
     if (mt.flags & kLast) {
       if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
