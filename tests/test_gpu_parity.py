@@ -468,6 +468,40 @@ def test_decode_scale_sign(oracle_mod, consumer, scale):
     _assert_close(out.cpu(), ref, torch.bfloat16, f"decode {consumer} scale={scale}")
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_prefill_edge_chunks(oracle_mod, prefill_consumer, dtype):
+    # sequences with no query token beside ones that have some; chunks of exactly one 64-key tile,
+    # one past it, exactly one 256-row unit (g = 4: 64 tokens) and one past it; whole prompts
+    # (context = chunk) and a chunk whose context ends on a block boundary
+    ctx = [50, 64, 65, 128, 129, 256, 300, 16]
+    nq = [0, 64, 65, 64, 65, 256, 0, 16]
+    case, q, q_start = _prefill_case(ctx, nq, 8, 2, 128, 16, dtype, 670)
+    ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                             case.scale, n_threads=0)
+    dev = case.to("cuda")
+    out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                         max_context_len=max(ctx), max_q_len=max(nq), scale=case.scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _assert_close(out.cpu(), ref, dtype, f"prefill edge chunks {prefill_consumer}")
+
+
+def test_prefill_without_queries_and_empty_decode_batch():
+    # every sequence contributes context but no query token: nothing to compute, no error
+    case, q, q_start = _prefill_case([40, 7], [0, 0], 8, 2, 64, 16, torch.bfloat16, 671)
+    dev = case.to("cuda")
+    q0 = torch.empty((0, 8, 64), dtype=torch.bfloat16, device="cuda")
+    out = api.pa_prefill(q0, q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
+                         max_context_len=40, max_q_len=0)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 8, 64)
+    # a decode batch of no sequence
+    case2 = W.paged_case("s0", [5], 8, 2, 64, 16, torch.bfloat16, 672).to("cuda")
+    out2 = api.pa_decode(case2.q[:0], case2.k_cache, case2.v_cache, case2.block_tables[:0], case2.context_lens[:0],
+                         max_context_len=5)
+    torch.cuda.synchronize()
+    assert out2.shape == (0, 8, 64)
+
+
 def test_prefill_single_tokens_match_decode():
     case = W.gqa8k_bf16(S=32)
     dev = case.to("cuda")
