@@ -19,7 +19,8 @@
  * Conventions for every entry point below.
  *   - Tensors are dense, row-major, contiguous.  "device" pointers point to memory the caller
  *     allocated on the current CUDA device; "host" pointers to host memory.  The library never
- *     takes ownership of a caller's buffer and never allocates device memory.
+ *     takes ownership of a caller's buffer and allocates no device buffers (scratch is a
+ *     caller-provided workspace; pa_step_create creates CUDA streams, events and graphs only).
  *   - Device pointers must be 16-byte aligned.
  *   - Device work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and
  *     runs asynchronously: a return of PA_OK means the arguments were valid and the kernels were
@@ -210,7 +211,14 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
  *   q_start       device [S+1] int32, non-decreasing, q_start[0] = 0
  *   k_cache, v_cache, block_tables, context_lens, B, n_blocks, max_blocks_per_seq: as pa_decode
  *   max_q_len     host bound on every n_s
- *   workspace     device scratch of pa_prefill_workspace_size(...) bytes, 256-byte aligned
+ *   scale         any finite value (usually 1/sqrt(d))
+ *   workspace     device scratch of pa_prefill_workspace_size(...) bytes, 256-byte aligned; its
+ *                 error word (pa_workspace_error) has bit 1 set if a bounded wait gave up and
+ *                 bit 2 if a size was cut to its bound
+ *
+ * Kernel: tcgen05 tensor cores with the S and O accumulators and P in tensor memory (default);
+ * the environment variable PA_PREFILL_CONSUMER=mma_sync selects the mma.sync kernel instead.
+ * Both give the same results within the tolerance (P is carried as two 16-bit parts).
  */
 size_t pa_prefill_workspace_size(int S, int H, int Hk, int max_q_len);
 
