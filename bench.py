@@ -129,6 +129,16 @@ class Workload:
         tables, lens = self.mgr.build_block_tables(self.seqs, self.max_blocks, tables, lens)
         return slots, pairs, tables, lens
 
+    def touched_bytes(self, lens):
+        """Bytes a decode launch moves counting whole blocks (the last block's unused slots too) and
+        the split-K partials (fp32 m, l and o written by the decode kernel, read by the combine)."""
+        S, H, Hk, d, B, es, P = self.S, self.H, self.Hk, self.d, self.B, self.es, self.P
+        lens = [int(c) for c in lens]
+        blocks = sum(-(-c // B) for c in lens)
+        parts = sum(-(-c // P) for c in lens if c > P)          # partitions of split sequences
+        return (blocks * B * Hk * d * 2 * es + S * H * d * es * 2 + 4 * blocks + 4 * S
+                + 2 * parts * H * (d + 2) * 4)
+
     def step_bytes(self, lens, n_pairs):
         S, H, Hk, d, B, es = self.S, self.H, self.Hk, self.d, self.B, self.es
         lens = [int(c) for c in lens]
@@ -368,6 +378,7 @@ def run_pa(args, rank, world, local_rank):
     decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     step_bytes = statistics.mean(traj[i % n_traj]["step_bytes"] for i in range(K))
     decode_bytes = statistics.mean(traj[i % n_traj]["decode_bytes"] for i in range(K))
+    touched_bytes = round(statistics.mean(wl.touched_bytes(traj[i % n_traj]["lens_host"]) for i in range(n_traj)))
     kv_bytes = statistics.mean(traj[i % n_traj]["kv_bytes"] for i in range(K))
     copy_bytes = statistics.mean(traj[i % n_traj]["n_pairs"] * 2 * Hk * wl.B * d * wl.es * 2 for i in range(K))
     write_bytes = 2 * (S * Hk * d * wl.es * 2) + 8 * S
@@ -479,6 +490,8 @@ def run_pa(args, rank, world, local_rank):
             "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(args),
             "algorithmic_bytes_per_launch": decode_bytes,
+            "touched_bytes_per_launch": touched_bytes,
+            "touched_gbs": round(touched_bytes / (decode_ms * 1e-3) / 1e9, 2),
             "launch_ms": round(decode_ms, 5),
         },
         "clocks": clock_info,
