@@ -61,6 +61,8 @@ PINS = [
     lambda o: pins.test_swap_blocks_matches_index_copy(o, torch.bfloat16),
     lambda o: pins.test_prefill_identity_table_equals_causal_sdpa(o, torch.bfloat16, 4, 128, 16),
     lambda o: pins.test_prefill_single_token_equals_decode(o),
+    lambda o: pins.test_brute_force_tiny_decode(o),
+    lambda o: pins.test_brute_force_tiny_prefill(o),
 ]
 
 

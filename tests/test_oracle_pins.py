@@ -4,6 +4,7 @@ routine and the block-wise formulation -- never against the oracle itself.
 Each test names the passage it follows (page title, section, equation).
 """
 import math
+import random
 
 import pytest
 import torch
@@ -351,3 +352,79 @@ def test_prefill_single_token_equals_decode(oracle_mod):
     od2 = oracle_mod.decode(q[q_start[1] + 3: q_start[1] + 4].expand(4, -1, -1).contiguous(), case.k_cache,
                             case.v_cache, case.block_tables, lens2)
     assert torch.allclose(o[q_start[1] + 3], od2[1], atol=1e-13, rtol=0)
+
+
+def _brute_layout(rnd, lens, Hk, d, B):
+    """A tiny paged cache in plain Python: blocks at shuffled physical ids, fp32-exact values."""
+    nb = [-(-c // B) for c in lens]
+    n_blocks = sum(nb) + 2
+    phys = list(range(n_blocks))
+    rnd.shuffle(phys)
+    kc = torch.full((n_blocks, Hk, B, d), float("nan"))
+    vc = torch.full((n_blocks, Hk, B, d), float("nan"))
+    tables = torch.full((len(lens), max(max(nb), 1)), -1, dtype=torch.int32)
+    i = 0
+    for s, c in enumerate(lens):
+        for j in range(nb[s]):
+            tables[s, j] = phys[i]
+            i += 1
+        for t in range(c):
+            p = int(tables[s, t // B])
+            for kh in range(Hk):
+                for e in range(d):
+                    kc[p, kh, t % B, e] = rnd.randint(-8, 8) / 4.0
+                    vc[p, kh, t % B, e] = rnd.randint(-8, 8) / 4.0
+    return kc, vc, tables
+
+
+def _brute_attend(qv, kc, vc, table, kh, n_keys, B, scale):
+    xs = []
+    for t in range(n_keys):
+        p, o = int(table[t // B]), t % B
+        xs.append(scale * sum(float(qv[e]) * float(kc[p, kh, o, e]) for e in range(len(qv))))
+    m = max(xs)
+    w = [math.exp(x - m) for x in xs]
+    z = sum(w)
+    return [sum(w[t] * float(vc[int(table[t // B]), kh, t % B, e]) for t in range(n_keys)) / z
+            for e in range(len(qv))]
+
+
+def test_brute_force_tiny_decode(oracle_mod):
+    # every (d <= 4, c <= 5, B in {1, 2}, g in {1, 2}) shape class, expanded by plain Python loops
+    rnd = random.Random(2024)
+    for trial in range(40):
+        d, B, g, Hk = rnd.randint(1, 4), rnd.choice([1, 2]), rnd.choice([1, 2]), rnd.choice([1, 2])
+        lens = [rnd.randint(1, 5) for _ in range(rnd.randint(1, 3))]
+        kc, vc, tables = _brute_layout(rnd, lens, Hk, d, B)
+        H = Hk * g
+        q = torch.tensor([[[rnd.randint(-8, 8) / 4.0 for _ in range(d)] for _ in range(H)] for _ in lens])
+        scale = rnd.choice([1.0, 0.5, 0.7])
+        o = oracle_mod.decode(q, kc, vc, tables, torch.tensor(lens, dtype=torch.int32), scale=scale)
+        for s, c in enumerate(lens):
+            for h in range(H):
+                ref = _brute_attend(q[s, h].tolist(), kc, vc, tables[s], h // g, c, B, scale)
+                for e in range(d):
+                    assert abs(float(o[s, h, e]) - ref[e]) <= 1e-12 * (1 + abs(ref[e])), (trial, s, h, e)
+
+
+def test_brute_force_tiny_prefill(oracle_mod):
+    # the token at position p = c - n + i attends to keys 0 .. p (plain Python loops)
+    rnd = random.Random(2025)
+    for trial in range(30):
+        d, B, g, Hk = rnd.randint(1, 4), rnd.choice([1, 2]), rnd.choice([1, 2]), 1
+        lens = [rnd.randint(1, 5) for _ in range(rnd.randint(1, 3))]
+        nq = [rnd.randint(0, c) for c in lens]
+        kc, vc, tables = _brute_layout(rnd, lens, Hk, d, B)
+        H = Hk * g
+        T = sum(nq)
+        q = torch.tensor([[[rnd.randint(-8, 8) / 4.0 for _ in range(d)] for _ in range(H)] for _ in range(T)])
+        q_start = torch.tensor([0] + [sum(nq[:i + 1]) for i in range(len(nq))], dtype=torch.int32)
+        o = oracle_mod.prefill(q.reshape(T, H, d), q_start, kc, vc, tables, torch.tensor(lens, dtype=torch.int32),
+                               scale=1.0)
+        for s, c in enumerate(lens):
+            for i in range(nq[s]):
+                row, pos = int(q_start[s]) + i, c - nq[s] + i
+                for h in range(H):
+                    ref = _brute_attend(q[row, h].tolist(), kc, vc, tables[s], h // g, pos + 1, B, 1.0)
+                    for e in range(d):
+                        assert abs(float(o[row, h, e]) - ref[e]) <= 1e-12 * (1 + abs(ref[e])), (trial, s, i, h)
