@@ -126,7 +126,10 @@ pa_status pa_decode_noalloc(void* out, pa_dtype out_dtype, const void* query, co
                             int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
                             void* stream);
 
-/* Partition size (tokens) that pa_decode uses for these arguments when given 0. */
+/* Partition size (tokens) that pa_decode uses for these arguments when given 0: the largest of
+ * 8192, 4096, ..., 256 with at least six units per SM of the current device when every sequence
+ * is max_context_len long, and no larger than the power of two that holds max_context_len
+ * (else 128). */
 int pa_decode_default_partition(int S, int Hk, int max_context_len);
 
 /* Copies the error word of a decode workspace to *flags (host) after synchronising `stream`.

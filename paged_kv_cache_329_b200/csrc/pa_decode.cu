@@ -108,7 +108,7 @@ WsLayout ws_layout(int S, int H, int Hk, int d, int max_parts) {
 // the persistent grid ends on short units.  Positions inside a group come from atomic cursors;
 // the order of units does not change any result (each unit's arithmetic is independent of it, and
 // partitions are merged in index order).
-constexpr int kBuckets = 64;
+constexpr int kBuckets = 128;
 
 __device__ __forceinline__ int tile_bucket(int ntok, int P) {
   const int tiles = (ntok + kTileTokens - 1) / kTileTokens;  // 0 .. P/64
@@ -1164,12 +1164,23 @@ cudaError_t dispatch_16bit(int d, int g, const CUtensorMap& tk, const CUtensorMa
 }
 
 int default_partition(int S, int Hk, int max_context_len) {
-  // Longer partitions mean fewer partial states to write and merge; the longest-first unit order
-  // keeps the persistent grid balanced as long as there are several units per CTA.  Measured on
-  // B200 (gqa8k_bf16, long_bf16): 1024 beats 512 and 256 by 5-15 %.
+  // Longer partitions mean fewer partial states to write and merge and fewer unit start-ups; the
+  // longest-first unit order keeps the persistent grid balanced while there are enough units per
+  // CTA.  The count below is an upper bound (every sequence at max_context_len), so the bar is six
+  // per SM.  Measured on B200 (fraction of the HBM copy peak): gqa8k 0.956 / 0.980 / 0.991 / 1.009
+  // at P = 1024 / 2048 / 4096 / 8192; long-context (16 seqs, 16-32 k tokens, B 16) 0.939 / 0.953 /
+  // 0.976 at 1024 / 2048 / 4096 but 0.813 at 8192 (about 384 actual units for 296 CTAs).
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  // No longer than the smallest of them that holds the longest context: beyond it nothing splits
+  // any more, and the shared-prefix workload (contexts ~1.1-1.4 k) measured 0.995 at 2048 but 0.98
+  // at 8192.
   const long long pairs = static_cast<long long>(S) * Hk;
-  for (int P : {1024, 512, 256})
-    if (pairs * ((max_context_len + P - 1) / P) >= 4 * 148) return P;
+  for (int P : {8192, 4096, 2048, 1024, 512, 256})
+    if (pairs * ((max_context_len + P - 1) / P) >= 6LL * sms && (P / 2 < max_context_len || P == 256)) return P;
   return 128;
 }
 
