@@ -140,13 +140,19 @@ __global__ void __launch_bounds__(kThreads) swap_blocks_kernel(uint4* __restrict
   }
 }
 
+// Grid for a grid-stride loop over work_items, per_block of them per CTA and round: at most 8 CTAs
+// per SM, and, when that takes several rounds, the smallest grid that needs the same number of
+// rounds, so that every CTA does the same number (2048 block copies on 1184 CTAs would leave half
+// of them idle for the second round; on 1024 CTAs each does two).
 int grid_for(long long work_items, int per_block) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long want = (work_items + per_block - 1) / per_block;
   const long long cap = static_cast<long long>(sms) * 8;
-  return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+  if (want <= cap) return static_cast<int>(want < 1 ? 1 : want);
+  const long long rounds = (want + cap - 1) / cap;
+  return static_cast<int>((want + rounds - 1) / rounds);
 }
 
 pa_status check_common(const void* kc, const void* vc, int Hk, int d, int B, int n_blocks, pa_dtype dtype,
