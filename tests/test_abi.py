@@ -81,3 +81,16 @@ def test_cache_ops_reject_bad_arguments(lib):
     assert lib.pa_copy_blocks(1 << 12, (1 << 12) + 4, 1 << 12, 1, 2, 128, 16, 8, 2, None) == api.PA_ERR_INVALID_ARG
     assert lib.pa_copy_blocks(1 << 12, 1 << 12, 1 << 12, 0, 2, 128, 16, 8, 2, None) == api.PA_OK  # nothing to do
     assert lib.pa_combine(1 << 12, 0, 1 << 12, 1 << 12, 1 << 12, 1 << 12, 2, 4, 80, 3, 64, None) == api.PA_ERR_UNSUPPORTED
+
+
+def test_default_partition_picks():
+    # the largest of 8192 .. 256 with six units per SM (148 SMs without a device) at the length
+    # bound, no larger than the power of two that holds the longest context; else 128
+    from paged_kv_cache_329_b200 import api
+    assert api.default_partition(256, 8, 8300) == 8192     # gqa8k: 2048 (seq, kv head) pairs
+    assert api.default_partition(16, 8, 33000) == 4096     # long context: 8192 would leave 640 units
+    assert api.default_partition(64, 40, 2200) == 4096     # 13B MHA: contexts <= 2200, no split
+    assert api.default_partition(128, 8, 1400) == 2048     # shared prefix
+    assert api.default_partition(256, 8, 100) == 256       # short contexts: one partition each
+    assert api.default_partition(4, 8, 300) == 128         # few pairs: split for parallelism
+    assert api.default_partition(1, 1, 5000) == 128
