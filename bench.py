@@ -401,9 +401,13 @@ def run_pa(args, rank, world, local_rank):
     e2e_bytes = 0
     stream = torch.cuda.current_stream()
 
+    host_s = []
+
     def prepare(st):
         nonlocal e2e_bytes
+        t_host = time.perf_counter()
         _, pr, _, ln = wl.host_step(st.h_slots, None, st.h_tables, st.h_lens)
+        host_s.append(time.perf_counter() - t_host)
         st.set_pairs(pr)
         c_sum, nb_sum = int(ln.sum()), int(((ln + (B - 1)) // B).sum())
         e2e_bytes += (c_sum * Hk * d * 2 * es + S * H * d * es * 2 + 4 * nb_sum + 4 * S
@@ -422,6 +426,7 @@ def run_pa(args, rank, world, local_rank):
 
     e2e_run(2)  # warm-up (also grows every sequence by two tokens)
     e2e_bytes = 0
+    host_s.clear()
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -502,6 +507,7 @@ def run_pa(args, rank, world, local_rank):
             "d2h_bytes_per_step": d2h // max(e2e_steps, 1),
             "steps": e2e_steps,
             "ms_per_step": round(e2e_ms / e2e_steps, 5),
+            "host_block_manager_ms": round(1e3 * statistics.median(host_s), 5) if host_s else None,
             "note": "per step: host block manager (prepared while the GPU runs the previous step), H2D "
                     "of the step's inputs from pinned memory, one replay of the captured kernels "
                     "(copy_blocks, cache_write, decode), D2H of o; the copies run on copy streams beside the "

@@ -24,6 +24,7 @@ struct pa_alloc {
   std::vector<int32_t> ref;   // reference count per physical block (0 = free)
   std::vector<int32_t> free;  // LIFO stack of free ids; back() is handed out next
   std::unordered_map<int32_t, Seq> seqs;
+  std::vector<std::vector<int32_t>> spare;  // table storage of freed sequences, reused by new ones
   int32_t next_seq = 0;
 };
 
@@ -40,6 +41,17 @@ int32_t take_block(pa_alloc* a) {  // caller checked that the stack is not empty
 
 void release(pa_alloc* a, int32_t b) {  // caller checked allocated(a, b)
   if (--a->ref[b] == 0) a->free.push_back(b);
+}
+
+// An empty table for a new sequence, taken from freed sequences' storage when there is some (a
+// serving loop forks and frees a batch of sequences every step; this keeps that free of
+// allocations once the pool has warmed up).
+std::vector<int32_t> fresh_table(pa_alloc* a) {
+  if (a->spare.empty()) return {};
+  std::vector<int32_t> t = std::move(a->spare.back());
+  a->spare.pop_back();
+  t.clear();
+  return t;
 }
 
 }  // namespace
@@ -59,6 +71,7 @@ pa_alloc* pa_alloc_create(int n_blocks, int B) {
   a->n_blocks = n_blocks;
   a->B = B;
   a->ref.assign(n_blocks, 0);
+  a->seqs.reserve(1024);
   a->free.resize(n_blocks);
   for (int i = 0; i < n_blocks; ++i) a->free[i] = n_blocks - 1 - i;  // back() == 0
   pa::ok();
@@ -96,7 +109,9 @@ int pa_alloc_num_free(const pa_alloc* a) { return a ? static_cast<int>(a->free.s
 pa_status pa_seq_create(pa_alloc* a, int32_t* seq_id) {
   if (!a || !seq_id) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_create: null argument");
   const int32_t id = a->next_seq++;
-  a->seqs.emplace(id, pa_alloc::Seq{});
+  pa_alloc::Seq s;
+  s.table = fresh_table(a);
+  a->seqs.emplace(id, std::move(s));
   *seq_id = id;
   return pa::ok();
 }
@@ -105,7 +120,10 @@ pa_status pa_seq_fork(pa_alloc* a, int32_t parent, int32_t* child) {
   if (!a || !child) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_fork: null argument");
   auto it = a->seqs.find(parent);
   if (it == a->seqs.end()) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_fork: unknown sequence %d", parent);
-  pa_alloc::Seq copy = it->second;
+  pa_alloc::Seq copy;
+  copy.table = fresh_table(a);
+  copy.table.assign(it->second.table.begin(), it->second.table.end());
+  copy.n_tokens = it->second.n_tokens;
   for (int32_t b : copy.table) ++a->ref[b];
   const int32_t id = a->next_seq++;
   a->seqs.emplace(id, std::move(copy));
@@ -118,6 +136,7 @@ pa_status pa_seq_free(pa_alloc* a, int32_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_free: unknown sequence %d", seq_id);
   for (int32_t b : it->second.table) release(a, b);
+  if (a->spare.size() < 4096) a->spare.push_back(std::move(it->second.table));
   a->seqs.erase(it);
   return pa::ok();
 }
