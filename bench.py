@@ -42,6 +42,7 @@ from paged_kv_cache_329_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode-attn effective KV GB/s (% of B200 HBM peak); seqs/s per step"
 L2_BYTES = 126e6   # B200 L2
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal bandwidth (about 8 TB/s), beside the measured copy peak
 E2E_DEPTH = 3      # decode steps in flight in the end-to-end leg
 
 
@@ -59,6 +60,12 @@ WORKLOADS = {
                                     "a 1024-token prompt (64 blocks at ref count 4), tails U[0,256]; every step "
                                     "each sequence forks from a seeded parent among its request's 4, so shared "
                                     "partial tail blocks are copied on write"),
+    "shared_prefix_partial_bf16": dict(S=128, H=32, Hk=8, d=128, B=16, dtype=torch.bfloat16, lens=None,
+                                       desc="shared-prefix sampling with a partial last prompt block, bf16: 32 "
+                                            "requests x 4 sequences share a 1031-token prompt (64 full blocks and "
+                                            "one of 7 tokens, all at ref count 4) and start generating; the first "
+                                            "step copies the partial block for 3 of each request's 4 sequences, "
+                                            "then beam-style forks as in the shared-prefix workload"),
     "tiny_fp32": dict(S=4, H=8, Hk=8, d=64, B=16, dtype=torch.float32,
                       lens=lambda: W.lens_uniform(W.generator(1), 4, 1, 200),
                       desc="tiny fp32 paged decode: 4 seqs, 8 q heads = 8 kv heads, d=64, B=16, context U[1,200]"),
@@ -71,11 +78,16 @@ WORKLOADS = {
 class Workload:
     """Sequences in a native block manager over a shuffled pool, random K/V in HBM."""
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0, seqs=0):
         cfg = dict(WORKLOADS[name])
         if block_size:
             cfg["B"] = block_size
             cfg["desc"] = cfg["desc"].replace("B=16", f"B={block_size}")
+        if seqs:       # the first `seqs` sequences only (a smaller case of the same workload, for profiling)
+            lens_fn = cfg["lens"]
+            cfg["lens"] = (lambda: lens_fn()[:seqs]) if lens_fn else None
+            cfg["S"] = seqs
+            cfg["desc"] += f" (first {seqs} sequences only)"
         self.name, self.cfg = name, cfg
         self.S, self.H, self.Hk, self.d, self.B, self.dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
         self.es = torch.finfo(self.dtype).bits // 8
@@ -154,8 +166,10 @@ class SharedPrefixWorkload(Workload):
 
     REQUESTS, WIDTH, PROMPT, TAIL_MAX = 32, 4, 1024, 256
 
-    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
+    def __init__(self, name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0, seqs=0):
         self.rnd = torch.Generator().manual_seed(4 + seed_offset)
+        if seqs:
+            raise ValueError("the shared-prefix workloads keep their 32 requests x 4 sequences")
         super().__init__(name, device, seed_offset, growth_steps + 64, partition, block_size)
 
     def _lengths(self):
@@ -200,9 +214,18 @@ class SharedPrefixWorkload(Workload):
         return len(used) * self.Hk * self.B * self.d * 2 * self.es
 
 
-def make_workload(name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0):
-    cls = SharedPrefixWorkload if name == "shared_prefix_bf16" else Workload
-    return cls(name, device, seed_offset, growth_steps, partition, block_size)
+class SharedPrefixPartialWorkload(SharedPrefixWorkload):
+    """The shared-prefix workload with a 1031-token prompt (its last block holds 7 tokens and is
+    shared by the request's 4 sequences) and no generated tokens yet: the first step's writes copy
+    that block for 3 of the 4 sequences, and the last one writes into it in place."""
+
+    PROMPT, TAIL_MAX = 1031, 0
+
+
+def make_workload(name, device, seed_offset=0, growth_steps=0, partition=0, block_size=0, seqs=0):
+    cls = {"shared_prefix_bf16": SharedPrefixWorkload,
+           "shared_prefix_partial_bf16": SharedPrefixPartialWorkload}.get(name, Workload)
+    return cls(name, device, seed_offset, growth_steps, partition, block_size, seqs)
 
 
 def load_peaks():
@@ -217,7 +240,7 @@ def load_peaks():
 def profiled_traffic(args):
     """DRAM bytes per decode launch from the committed ncu summary, if its source hash matches and
     the run is the workload it was captured on (gqa8k_bf16, library-default partition and B)."""
-    if args.workload != "gqa8k_bf16" or args.partition or args.block_size:
+    if args.workload != "gqa8k_bf16" or args.partition or args.block_size or args.seqs:
         return None
     path = os.path.join(ROOT, "profiles", "decode_kernel_gqa8k_bf16.md")
     src = os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", "pa_decode.cu")
@@ -316,10 +339,10 @@ def run_pa(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     K, Wm = args.steps, args.warmup
-    e2e_steps = min(K, args.e2e_steps)
-    n_traj = 32 if args.workload == "shared_prefix_bf16" else 1
+    e2e_steps = args.e2e_steps
+    n_traj = 32 if args.workload.startswith("shared_prefix") else 1
     wl = make_workload(args.workload, dev, seed_offset=rank, growth_steps=e2e_steps + Wm + n_traj + 2,
-                       partition=args.partition, block_size=args.block_size)
+                       partition=args.partition, block_size=args.block_size, seqs=args.seqs)
     S, H, Hk, d = wl.S, wl.H, wl.Hk, wl.d
     gen = torch.Generator(device=dev).manual_seed(99 + rank)
     q = torch.randn((S, H, d), generator=gen, device=dev).to(wl.dtype)
@@ -333,22 +356,24 @@ def run_pa(args, rank, world, local_rank):
     for st in traj:
         st["decode_bytes"], st["step_bytes"], st["kv_bytes"] = wl.step_bytes(st["lens_host"], st["n_pairs"])
     max_parts = -(-wl.max_c // wl.P)
-    launches = [2 + (1 if max_parts > 1 else 0) + 1 + (1 if st["n_pairs"] else 0) for st in traj]
+    launches = [2 + (1 if max_parts > 1 else 0) for st in traj]      # prologue, decode, combine
 
-    def device_step(st, evs=None):
-        if evs is not None:
-            evs[0].record()
+    def device_step(st):
+        """The step as one call: copies, writes and the plan in one kernel, then decode (and combine)."""
+        api.pa_decode_step(q, wl.k_cache, wl.v_cache, st["tables"], st["lens"], key, val, st["slots"], st["pairs"],
+                           max_context_len=wl.max_c, out=out, partition_size=wl.P, workspace=wl.workspace)
+
+    def separate_calls(st, evs):
+        """The same step as three calls, timed call by call (the decode call gives the roofline)."""
+        evs[0].record()
         if st["n_pairs"]:
             api.pa_copy_blocks(wl.k_cache, wl.v_cache, st["pairs"])
-        if evs is not None:
-            evs[1].record()
+        evs[1].record()
         api.pa_cache_write(wl.k_cache, wl.v_cache, key, val, st["slots"])
-        if evs is not None:
-            evs[2].record()
+        evs[2].record()
         api.pa_decode(q, wl.k_cache, wl.v_cache, st["tables"], st["lens"], max_context_len=wl.max_c, out=out,
                       partition_size=wl.P, workspace=wl.workspace)
-        if evs is not None:
-            evs[3].record()
+        evs[3].record()
 
     def barrier():
         if world > 1:
@@ -359,20 +384,36 @@ def run_pa(args, rank, world, local_rank):
         device_step(traj[i % n_traj])
     torch.cuda.synchronize()
     assert api.workspace_error(wl.workspace) == 0, "decode reported an error"
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    step_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record()
     for i in range(K):
-        device_step(traj[i % n_traj], evs[i])
+        step_evs[i][0].record()
+        device_step(traj[i % n_traj])
+        step_evs[i][1].record()
     stop.record()
     torch.cuda.synchronize()
     barrier()
-    t_wall1 = time.time()
-    clocks.mark(t_wall0, t_wall1)
+    clocks.mark(t_wall0, time.time())
     total_ms = start.elapsed_time(stop)
+    step_times = sorted(e[0].elapsed_time(e[1]) for e in step_evs)
+
+    # the same K steps as separate calls: per-call times, and the decode call's roofline
+    for i in range(Wm):
+        separate_calls(traj[i % n_traj], [torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(K):
+        separate_calls(traj[i % n_traj], evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clocks.mark(t_wall0, time.time())
+    separate_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)
     copy_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     write_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -441,8 +482,8 @@ def run_pa(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
     clock_info = clocks.finish()
 
-    total_ms, e2e_ms, decode_ms, copy_ms, write_ms = reduce_max([total_ms, e2e_ms, decode_ms, copy_ms, write_ms],
-                                                                world, dev)
+    total_ms, e2e_ms, decode_ms, copy_ms, write_ms, separate_ms = reduce_max(
+        [total_ms, e2e_ms, decode_ms, copy_ms, write_ms, separate_ms], world, dev)
     if rank != 0:
         return None
 
@@ -458,6 +499,9 @@ def run_pa(args, rank, world, local_rank):
         "steps": K,
         "warmup": Wm,
         "ms_per_step": round(ms_per_step, 5),
+        "step_ms_spread": {"min": round(step_times[0], 5), "median": round(statistics.median(step_times), 5),
+                           "max": round(step_times[-1], 5), "of": len(step_times),
+                           "note": "CUDA events around each timed step (one pa_decode_step call)"},
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -472,27 +516,33 @@ def run_pa(args, rank, world, local_rank):
             "l2": (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush"
                    if kv_bytes > L2_BYTES else
                    f"warm: the {kv_bytes / 1e6:.1f} MB of K/V read per step fit in L2 (no flush)"),
-            "step": "host block manager -> pa_copy_blocks -> pa_cache_write -> pa_decode (plan, decode, combine)",
+            "step": "host block manager -> pa_decode_step (COW copies, slot writes and the decode plan in one "
+                    "kernel, then decode and combine)",
             "step_bytes": round(step_bytes),
             "cow_pairs_per_step": n_pairs,
             "trajectory_steps": n_traj,
             **({"unique_kv_bytes_step0": wl.unique_kv_bytes(traj[0]["tables"].cpu(), lens),
                 "logical_kv_bytes_step0": traj[0]["kv_bytes"]} if hasattr(wl, "unique_kv_bytes") else {}),
         },
-        "kernel_ms": {"copy_blocks": round(copy_ms, 5), "cache_write": round(write_ms, 5),
-                      "decode": round(decode_ms, 5)},
+        "kernel_ms": {"step": round(ms_per_step, 5), "decode": round(decode_ms, 5),
+                      "step_over_decode": round(ms_per_step / decode_ms, 4),
+                      "separate_calls": {"copy_blocks": round(copy_ms, 5), "cache_write": round(write_ms, 5),
+                                         "decode": round(decode_ms, 5), "step": round(separate_ms, 5)}},
         "kernel_gbs": {"copy_blocks": round(copy_bytes / (copy_ms * 1e-3) / 1e9, 2) if copy_bytes else None,
                        "cache_write": round(write_bytes / (write_ms * 1e-3) / 1e9, 2)},
         "seqs_per_s": round(S * world / (ms_per_step * 1e-3), 1),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "pct_of_nominal_hbm": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "roofline": {
             "bound": "hbm",
-            "kernel": "pa_decode (plan + decode_kernel + combine, CUDA events around the call)",
+            "kernel": "pa_decode (plan + decode_kernel + combine, CUDA events around each of K calls)",
             "achieved": round(achieved, 2),
             "peak": peak,
             "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "nominal_gbs": NOMINAL_HBM_GBS,
             "traffic": profiled_traffic(args),
             "algorithmic_bytes_per_launch": decode_bytes,
             "touched_bytes_per_launch": touched_bytes,
@@ -510,7 +560,8 @@ def run_pa(args, rank, world, local_rank):
             "host_block_manager_ms": round(1e3 * statistics.median(host_s), 5) if host_s else None,
             "note": "per step: host block manager (prepared while the GPU runs the previous step), H2D "
                     "of the step's inputs from pinned memory, one replay of the captured kernels "
-                    "(copy_blocks, cache_write, decode), D2H of o; the copies run on copy streams beside the "
+                    "(pa_decode_step: copies, writes and plan, decode, combine), D2H of o; the copies run on "
+                    "copy streams beside the "
                     "neighbouring steps' kernels; every step's output is read back (at most "
                     f"{E2E_DEPTH} steps in flight)",
         },
@@ -712,8 +763,9 @@ def run_prefill(args, rank, world, local_rank):
 
 def run_cache_ops(args, rank, world, local_rank):
     """The copy-on-write copy and the slot-mapped write at sizes where they are bandwidth-bound:
-    1024 (src, dst) pairs of gqa8k-shaped blocks (8 kv heads x 16 tokens x 128 dims, bf16) and
-    65536 new tokens written through a random slot mapping into a 65536-block pool."""
+    4096 (src, dst) pairs of gqa8k-shaped blocks (8 kv heads x 16 tokens x 128 dims, bf16; 256 MiB
+    written, twice the L2, so the copies' writes reach DRAM within the launch) and 65536 new tokens
+    written through a random slot mapping into a 65536-block pool."""
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     n_blocks, Hk, B, d, dt = 65536, 8, 16, 128, torch.bfloat16
@@ -722,12 +774,13 @@ def run_cache_ops(args, rank, world, local_rank):
     vc = torch.randn((n_blocks, Hk, B, d), generator=gen, device=dev).to(dt)
     g = torch.Generator().manual_seed(32)
     perm = torch.randperm(n_blocks, generator=g)
-    pairs = torch.stack([perm[:1024], perm[1024:2048]], 1).to(torch.int32).to(dev)
+    n_pairs = 4096
+    pairs = torch.stack([perm[:n_pairs], perm[n_pairs:2 * n_pairs]], 1).to(torch.int32).to(dev)
     T = 65536
     slots = torch.randperm(n_blocks * B, generator=g)[:T].to(dev)
     key = torch.randn((T, Hk, d), generator=gen, device=dev).to(dt)
     val = torch.randn((T, Hk, d), generator=gen, device=dev).to(dt)
-    copy_bytes = 1024 * 2 * (Hk * B * d * 2) * 2
+    copy_bytes = n_pairs * 2 * (Hk * B * d * 2) * 2
     write_bytes = 2 * (T * Hk * d * 2 * 2) + 8 * T
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for _ in range(args.warmup):
@@ -758,7 +811,7 @@ def run_cache_ops(args, rank, world, local_rank):
             "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round((copy_ms + write_ms) / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "1024 COW pairs of 8x16x128 bf16 blocks + 65536 slot writes (8x128 bf16 K and V)",
+            "config": {"workload": f"{n_pairs} COW pairs of 8x16x128 bf16 blocks + 65536 slot writes (8x128 bf16 K and V)",
                        "copy_bytes": copy_bytes, "write_bytes": write_bytes},
             "kernels": {"copy_blocks": {"GB/s": round(copy_gbs, 2), "frac": round(copy_gbs / world / peak, 4),
                                         "ms": round(copy_ms / args.steps, 5)},
@@ -779,7 +832,11 @@ def run_reference(args, rank, world):
     cfg = dict(WORKLOADS[args.workload])
     if args.block_size:
         cfg["B"] = args.block_size
-    lens = cfg["lens"]().tolist() if cfg["lens"] else [1024 + 128] * cfg["S"]   # shared prefix: prompt + mean tail
+    if cfg["lens"]:
+        lens = cfg["lens"]().tolist()
+    else:                                              # shared prefix: prompt + mean tail + the new token
+        wl_cls = SharedPrefixPartialWorkload if args.workload == "shared_prefix_partial_bf16" else SharedPrefixWorkload
+        lens = [wl_cls.PROMPT + wl_cls.TAIL_MAX // 2 + 1] * cfg["S"]
     S, H, Hk, d, B, dtype = (cfg[k] for k in ("S", "H", "Hk", "d", "B", "dtype"))
     es = torch.finfo(dtype).bits // 8
     cores = oracle.hardware_threads()
@@ -845,9 +902,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="pa", choices=["pa", "reference"])
     ap.add_argument("--workload", default="gqa8k_bf16", choices=sorted(WORKLOADS) + ["swap_bf16", "prefill_mixed_bf16", "cache_ops_bf16"])
-    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--partition", type=int, default=0, help="decode partition size in tokens (0 = library default)")
     ap.add_argument("--block-size", type=int, default=0, help="tokens per KV block (0 = the workload's own)")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="keep only the first N sequences of a decode workload (0 = all; a smaller case for ncu)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
