@@ -100,6 +100,33 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void
                     int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* One decode step on device-resident inputs: the copy-on-write block copies, then the slot-mapped
+ * write of the new tokens, then paged decode attention -- the order the pages give ("解决COW":
+ * copy the shared block before writing into the copy; "vllm" 2.2 Decode: the new token's K and V
+ * are stored, then attended over).  The result equals
+ *     pa_copy_blocks(k_cache, v_cache, pairs, n);  pa_cache_write(..., key, value, slot_mapping, T);
+ *     pa_decode(out, ...);
+ * in fewer launches: one kernel makes the copies, the writes and the decode's work plan (a block
+ * copy and every write into the copied block are made by the same CTA, copy first), and the
+ * decode kernels follow it by programmatic dependent launch and wait for all of it.
+ *
+ *   key, value     device [T][Hk][d] of kv_dtype: the new tokens
+ *   slot_mapping   device [T] int64, slot = block * B + offset (< 0: padding, skipped)
+ *   pairs          device [max_pairs][2] int32 (src, dst), destinations distinct and no
+ *                  destination also a source (as the block manager emits them)
+ *   n_pairs        device pointer to the number of pairs used (clamped to [0, max_pairs]), read by
+ *                  the kernel -- so one capture serves steps with different counts -- or NULL to
+ *                  use all max_pairs; max_pairs <= 8192
+ *   everything else: as pa_decode (workspace of pa_decode_workspace_size(...) bytes).
+ * Out-of-range block ids in pairs or slots are skipped as in pa_copy_blocks / pa_cache_write. */
+pa_status pa_decode_step(void* out, pa_dtype out_dtype, const void* query, void* k_cache, void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, const void* key,
+                         const void* value, const int64_t* slot_mapping, int T, const int32_t* pairs,
+                         const int32_t* n_pairs, int max_pairs, int S, int H, int Hk, int d, int B,
+                         int n_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                         pa_dtype kv_dtype, int partition_size, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
 /* Paged decode attention that allocates nothing and takes no workspace.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot call cudaMalloc: plugins
  * whose host process owns the whole device-memory budget and forbids allocations by libraries,
@@ -114,7 +141,9 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void
  * pa_decode with a caller-provided workspace, serves them).
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current) and caches it; make that first call before any stream capture.  Every
+ * that device current) and caches it for the device's current context; make that first call
+ * before any stream capture.  After a device reset (a new context) the next call looks the
+ * address up again, so that call too should come before any stream capture.  Every
  * call uses the same array, which keeps the last call's contents; the only fields that must
  * start from known values (the unit counter, the unit count and the error word) are reset by the
  * call's own first kernel.  Calls that overlap on the GPU (different streams, or different host

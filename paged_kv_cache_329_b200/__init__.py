@@ -17,6 +17,7 @@ from .api import (  # noqa: F401
     pa_combine,
     pa_copy_blocks,
     pa_decode,
+    pa_decode_step,
     pa_prefill,
     pa_swap_blocks,
     version,

@@ -38,6 +38,7 @@ SIGNATURES = {
     "pa_version": (ctypes.c_char_p, []),
     "pa_decode_workspace_size": (SZ, [I, I, I, I, I, I]),
     "pa_decode": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
+    "pa_decode_step": (I, [P, I, P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
     "pa_decode_noalloc": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P]),
     "pa_decode_default_partition": (I, [I, I, I]),
     "pa_prefill_workspace_size": (SZ, [I, I, I, I]),

@@ -93,6 +93,40 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, *, max_context_le
     return out
 
 
+def pa_decode_step(q, k_cache, v_cache, block_tables, context_lens, key, value, slot_mapping, pairs, *,
+                   max_context_len, n_pairs=None, scale=None, out=None, out_dtype=None, partition_size=0,
+                   workspace=None, stream=None):
+    """One decode step: copy-on-write copies, slot writes, then decode, in fewer launches; returns out.
+    pairs: int32 [max_pairs, 2] on the device; n_pairs: an int32 device tensor holding the count
+    used (or None: every row of pairs).  See pa_decode_step in include/pa.h."""
+    _cuda(q, k_cache, v_cache, block_tables, context_lens, key, value, slot_mapping, pairs)
+    S, H, d = q.shape
+    n_blocks, Hk, B, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape or q.dtype != k_cache.dtype or key.dtype != k_cache.dtype \
+            or value.dtype != k_cache.dtype:
+        raise ValueError("shape/dtype mismatch between q, key, value and the caches")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32 or pairs.dtype != torch.int32 \
+            or slot_mapping.dtype != torch.int64:
+        raise ValueError("block_tables, context_lens and pairs must be int32, slot_mapping int64")
+    if n_pairs is not None:
+        _cuda(n_pairs)
+        if n_pairs.dtype != torch.int32:
+            raise ValueError("n_pairs must be an int32 device tensor")
+    if out is None:
+        out = torch.empty((S, H, d), dtype=out_dtype or q.dtype, device=q.device)
+    _cuda(out)
+    if workspace is None:
+        workspace = alloc_workspace(S, H, Hk, d, max_context_len, partition_size, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(_native.load().pa_decode_step(
+        _ptr(out), DTYPE[out.dtype], _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        _ptr(key), _ptr(value), _ptr(slot_mapping), key.shape[0], _ptr(pairs), _ptr(n_pairs), pairs.numel() // 2,
+        S, H, Hk, d, B, n_blocks, block_tables.shape[1], int(max_context_len), float(scale), DTYPE[q.dtype],
+        int(partition_size), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def pa_prefill(q, q_start, k_cache, v_cache, block_tables, context_lens, *, max_context_len, max_q_len,
                scale=None, out=None, out_dtype=None, workspace=None, stream=None):
     """Causal paged attention for several query tokens per sequence (prefill chunks and decode tokens

@@ -119,51 +119,213 @@ __device__ __forceinline__ int tile_bucket(int ntok, int P) {
 
 constexpr int kPlanCache = 4096;  // lengths kept in shared memory between the two passes
 
+struct PlanSmem {
+  int count[kBuckets], cursor[kBuckets];
+  int c_cache[kPlanCache];
+};
+
+// Lists the units of one decode launch into items[] and resets the workspace header; run by one
+// whole CTA (any block size that is a multiple of 32).  Each bucket's start is an exclusive
+// prefix sum over the buckets from the longest down, taken by the first warp.
+__device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restrict__ lens, int S, int Hk, int P,
+                                           int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int nb = min(P / kTileTokens, kBuckets);
+  for (int b = tid; b < kBuckets; b += nt) sm.count[b] = 0;
+  __syncthreads();
+  bool clamped = false;
+  for (int s = tid; s < S; s += nt) {
+    const int raw = lens[s];
+    clamped |= raw > max_c;
+    const int c = min(max(raw, 0), max_c);
+    if (s < kPlanCache) sm.c_cache[s] = c;
+    const int f = max(1, (c + P - 1) / P) - 1;  // whole partitions before the last one
+    if (f > 0) atomicAdd(&sm.count[nb - 1], f * Hk);
+    atomicAdd(&sm.count[tile_bucket(c - f * P, P)], Hk);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // buckets nb-1, nb-2, ..., 0 in that order: lane l owns positions 4l .. 4l+3 of it
+    constexpr int kPer = kBuckets / 32;
+    int v[kPer], run = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int pos = tid * kPer + i;
+      v[i] = pos < nb ? sm.count[nb - 1 - pos] : 0;
+      run += v[i];
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
+    }
+    int excl = incl - run;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int pos = tid * kPer + i;
+      if (pos < nb) sm.cursor[nb - 1 - pos] = excl;
+      excl += v[i];
+    }
+    if (tid == 31) {
+      hdr[kHdrCounter] = 0;
+      hdr[kHdrNumItems] = incl;
+    }
+  }
+  __syncthreads();
+  for (int s = tid; s < S; s += nt) {
+    const int c = s < kPlanCache ? sm.c_cache[s] : min(max(lens[s], 0), max_c);
+    const int f = max(1, (c + P - 1) / P) - 1;
+    if (f > 0) {
+      const int base = atomicAdd(&sm.cursor[nb - 1], f * Hk);
+      for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+    }
+    const int base = atomicAdd(&sm.cursor[tile_bucket(c - f * P, P)], Hk);
+    for (int kh = 0; kh < Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | f);
+  }
+  const int any_clamped = __syncthreads_or(clamped);
+  if (tid == 0) hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ lens, int S, int Hk, int P,
                                                             int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
   // Let the decode grid start its set-up now; wait for earlier work on the stream (it may have
   // written the lengths) before reading anything.
   pa::grid_dependency_launch();
   pa::grid_dependency_wait();
-  __shared__ int count[kBuckets], cursor[kBuckets];
-  __shared__ int c_cache[kPlanCache];
-  const int tid = threadIdx.x;
-  const int nb = min(P / kTileTokens, kBuckets);
-  for (int b = tid; b < kBuckets; b += kPlanThreads) count[b] = 0;
-  __syncthreads();
-  bool clamped = false;
-  for (int s = tid; s < S; s += kPlanThreads) {
-    const int raw = lens[s];
-    clamped |= raw > max_c;
-    const int c = min(max(raw, 0), max_c);
-    if (s < kPlanCache) c_cache[s] = c;
-    const int f = max(1, (c + P - 1) / P) - 1;  // whole partitions before the last one
-    if (f > 0) atomicAdd(&count[nb - 1], f * Hk);
-    atomicAdd(&count[tile_bucket(c - f * P, P)], Hk);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int b = nb - 1; b >= 0; --b) {
-      cursor[b] = run;
-      run += count[b];
+  __shared__ PlanSmem sm;
+  build_plan(sm, lens, S, Hk, P, max_c, items, hdr);
+}
+
+// ---- step prologue: copy-on-write copies, slot writes and the plan in one launch ---------------
+// "解决COW" orders a shared block's copy before the write into the copy, and the decode reads the
+// cache after both.  CTA 0 builds the decode plan (it reads only the lengths).  Every other CTA
+// takes copy pairs p = blockIdx.x - 1, ... in steps of gridDim.x - 1: it copies the pair's K and
+// V block and then itself writes every new token whose slot lies in the destination block, so the
+// write follows the copy within one CTA.  Tokens whose block is no copy destination are written by
+// any CTA, one warp per token.  The decode kernels wait for this whole grid (griddepcontrol.wait).
+constexpr int kPrologueThreads = 256;
+using pa::kMaxStepPairs;
+
+struct PrologueArgs {
+  uint4* kc;
+  uint4* vc;
+  const uint4* key;
+  const uint4* value;
+  const int64_t* slots;
+  const int32_t* pairs;
+  const int32_t* n_pairs_dev;  // count on the device, or null: max_pairs
+  int T, max_pairs, Hk, chunks, B, n_blocks;
+  long long vec_per_block;     // 16-byte vectors per block and cache (Hk * B * d * e / 16)
+};
+
+// The rows of token n (slot = blk * B + off, blk in range) of key and value, by the given threads.
+__device__ __forceinline__ void write_token(const PrologueArgs& w, int n, long long blk, int off, int t0, int nt) {
+  const int per_token = w.Hk * w.chunks;
+  const uint4* ks = w.key + static_cast<long long>(n) * per_token;
+  const uint4* vs = w.value + static_cast<long long>(n) * per_token;
+  uint4* kd = w.kc + (blk * w.Hk * w.B + off) * w.chunks;
+  uint4* vd = w.vc + (blk * w.Hk * w.B + off) * w.chunks;
+  for (int v0 = t0; v0 < per_token; v0 += 4 * nt) {
+    uint4 kb[4], vb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * nt;
+      if (v < per_token) {
+        kb[u] = __ldg(ks + v);
+        vb[u] = __ldg(vs + v);
+      }
     }
-    hdr[kHdrCounter] = 0;
-    hdr[kHdrNumItems] = run;
-  }
-  __syncthreads();
-  for (int s = tid; s < S; s += kPlanThreads) {
-    const int c = s < kPlanCache ? c_cache[s] : min(max(lens[s], 0), max_c);
-    const int f = max(1, (c + P - 1) / P) - 1;
-    if (f > 0) {
-      const int base = atomicAdd(&cursor[nb - 1], f * Hk);
-      for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * nt;
+      if (v < per_token) {
+        const int kh = v / w.chunks, c = v - kh * w.chunks;
+        const long long o = static_cast<long long>(kh) * w.B * w.chunks + c;
+        kd[o] = kb[u];
+        vd[o] = vb[u];
+      }
     }
-    const int base = atomicAdd(&cursor[tile_bucket(c - f * P, P)], Hk);
-    for (int kh = 0; kh < Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | f);
   }
-  const int any_clamped = __syncthreads_or(clamped);
-  if (tid == 0) hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
+}
+
+__global__ void __launch_bounds__(kPrologueThreads) step_prologue_kernel(PrologueArgs w, const int32_t* __restrict__ lens,
+                                                                         int S, int Hk, int P, int max_c,
+                                                                         int2* __restrict__ items, int* __restrict__ hdr) {
+  // The previous step's kernels may still read blocks this step overwrites (a freed block can be
+  // a copy destination now), and its decode reads the workspace: wait for them before any write.
+  pa::grid_dependency_wait();
+  pa::grid_dependency_launch();
+  __shared__ union {
+    PlanSmem plan;
+    int32_t dst[kMaxStepPairs];
+  } sm;
+  __shared__ int n_mine;
+  __shared__ int mine[kPrologueThreads];
+  if (blockIdx.x == 0) {
+    build_plan(sm.plan, lens, S, Hk, P, max_c, items, hdr);
+    return;
+  }
+  const int n_pairs = w.n_pairs_dev ? min(max(*w.n_pairs_dev, 0), w.max_pairs) : w.max_pairs;
+  for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) sm.dst[i] = __ldg(w.pairs + 2 * i + 1);
+  __syncthreads();
+  const int workers = gridDim.x - 1, wid = blockIdx.x - 1;
+  // (a) block copies, each followed by the writes into its destination
+  for (int p = wid; p < n_pairs; p += workers) {
+    const int src = __ldg(w.pairs + 2 * p), dst = sm.dst[p];
+    if (src >= 0 && src < w.n_blocks && dst >= 0 && dst < w.n_blocks) {
+#pragma unroll 1
+      for (int cache = 0; cache < 2; ++cache) {
+        const uint4* sp = (cache ? w.vc : w.kc) + static_cast<long long>(src) * w.vec_per_block;
+        uint4* dp = (cache ? w.vc : w.kc) + static_cast<long long>(dst) * w.vec_per_block;
+        for (long long v0 = 0; v0 < w.vec_per_block; v0 += 8LL * kPrologueThreads) {
+          uint4 b[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const long long v = v0 + u * kPrologueThreads + threadIdx.x;
+            if (v < w.vec_per_block) b[u] = sp[v];
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const long long v = v0 + u * kPrologueThreads + threadIdx.x;
+            if (v < w.vec_per_block) dp[v] = b[u];
+          }
+        }
+      }
+    }
+    if (threadIdx.x == 0) n_mine = 0;
+    __syncthreads();  // the copy is complete (and visible to the CTA) before the writes below
+    for (int n = threadIdx.x; n < w.T; n += blockDim.x) {
+      const int64_t slot = __ldg(w.slots + n);
+      if (slot >= 0 && slot / w.B == dst) {
+        const int k = atomicAdd(&n_mine, 1);
+        if (k < kPrologueThreads) mine[k] = n;
+      }
+    }
+    __syncthreads();
+    const int cnt = min(n_mine, kPrologueThreads);
+    if (dst >= 0 && dst < w.n_blocks) {
+      for (int i = 0; i < cnt; ++i) {
+        const int n = mine[i];
+        const int64_t slot = __ldg(w.slots + n);
+        write_token(w, n, slot / w.B, static_cast<int>(slot % w.B), threadIdx.x, blockDim.x);
+      }
+    }
+    __syncthreads();
+  }
+  // (b) the other tokens, one warp each
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_warps = workers * (kPrologueThreads / 32);
+  for (int n = wid * (kPrologueThreads / 32) + warp; n < w.T; n += n_warps) {
+    const int64_t slot = __ldg(w.slots + n);
+    if (slot < 0) continue;
+    const int64_t blk = slot / w.B;
+    if (blk >= w.n_blocks) continue;
+    bool copied = false;
+    for (int i = lane; i < n_pairs && !copied; i += 32) copied = sm.dst[i] == blk;
+    if (__any_sync(0xffffffffu, copied)) continue;  // written by the CTA that copied its block
+    write_token(w, n, blk, static_cast<int>(slot - blk * w.B), lane, 32);
+  }
 }
 
 // ---- the decode kernel --------------------------------------------------------------------------
@@ -175,8 +337,7 @@ struct Cfg {
   static constexpr int kCH = D / kE;                          // chunks per row
   static constexpr int kPanelElems = 128 / kES;               // elements per 128-byte panel row
   static constexpr int kNPanel = D / kPanelElems;             // panels per row
-  static constexpr int kPanelBytes = kTileTokens * 128;       // one panel of one tile
-  static constexpr int kKVBytes = kNPanel * kPanelBytes;      // K (or V) tile
+  static constexpr int kKVBytes = kTileTokens * D * kES;     // K (or V) tile
   static constexpr int kStageBytes = 2 * kKVBytes;
   static constexpr int kStages = kNPanel == 1 ? 6 : 3;
   static constexpr int kQBytes = G * D * kES;
@@ -198,6 +359,26 @@ struct Cfg {
   static_assert(kPasses >= 1 && kTileTokens % (kConsumerWarps * kTPW) == 0, "tile/mapping mismatch");
   static_assert(kCH % kL == 0, "chunks must split evenly over lanes");
   static_assert(kQBytes % 16 == 0, "q rows must be whole 16-byte chunks");
+};
+
+// Shared-memory place of tile row t (0..63), 16-byte chunk c of a K or V tile.  A tile holds its
+// 64/B blocks one after the other; each block is one TMA box of B rows laid out panel by panel
+// (a panel = 128 bytes of every row, so d = 128 at 16 bits has 2 panels), and the 128-byte
+// swizzle puts chunk c of row t at chunk (c % 8) ^ (t % 8) of its 128-byte line, which keeps the
+// 8 rows that one ldmatrix phase reads on distinct banks.
+struct TileAddr {
+  int panel_stride;  // B * 128: from one panel of a block to the next
+  int blk_extra;     // B * 128 * (panels - 1): what a block adds beyond its B rows of 128 bytes
+  int log2b;
+  __device__ __forceinline__ TileAddr(int B, int n_panel) {
+    panel_stride = B * 128;
+    blk_extra = B * 128 * (n_panel - 1);
+    log2b = B == 8 ? 3 : (B == 16 ? 4 : 5);
+  }
+  __device__ __forceinline__ int row(int t) const { return t * 128 + (t >> log2b) * blk_extra; }
+  __device__ __forceinline__ int chunk(int t, int c) const {
+    return (c >> 3) * panel_stride + (((c & 7) ^ (t & 7)) << 4);
+  }
 };
 
 // Reduce-scatter of partial dot products over the L lanes of a token group: at each level with
@@ -323,6 +504,9 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
   const int ld_hi = lane >> 4;
   const int ldt_row = (lane >> 4) * 8 + (lane & 7);            // p.V: tiles (lo, hi dims) x (tok 0-7, tok 8-15)
   const int ldt_hi = (lane >> 3) & 1;
+  const TileAddr ta(a.B, C::kNPanel);
+  const int k_row = warp * 16 + ld_row, v_row = warp * 16 + ldt_row;
+  const int k_row_off = ta.row(k_row), v_row_off = ta.row(v_row);
 
   while (true) {
     if (!pa::mbar_wait(&full[stage], phase)) {
@@ -359,7 +543,7 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
       for (int k = 0; k < KS; ++k) {
         const int row = r0 + ld_row, c = 2 * k + ld_hi;
         uint32_t af[4];
-        pa::ldsm_x4(af, kbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+        pa::ldsm_x4(af, kbase + k_row_off + ta.chunk(row, c));
         M::run(sacc, af, bq[k]);
       }
       // ---- online softmax; this lane holds tokens gq, gq+8 for heads 2tq, 2tq+1 ----
@@ -416,7 +600,7 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
       for (int k = 0; k < KS; ++k) {
         const int row = r0 + ldt_row, c = 2 * k + ldt_hi;
         uint32_t af[4];
-        pa::ldsm_x4_trans(af, vbase + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+        pa::ldsm_x4_trans(af, vbase + v_row_off + ta.chunk(row, c));
         af[0] &= mask01;
         af[1] &= mask01;
         af[2] &= mask23;
@@ -628,11 +812,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         uint8_t* kdst = stages + stage * C::kStageBytes;
         uint8_t* vdst = kdst + C::kKVBytes;
         if (lane < nblk) {
+          // one box per (block, K or V): B rows x every panel (a 3-D box when there are several)
           const int y = (phys * a.Hk + kh) * a.B;
-#pragma unroll
-          for (int p = 0; p < C::kNPanel; ++p) {
-            pa::tma_load_2d(kdst + p * C::kPanelBytes + lane * a.B * 128, &tmK, p * C::kPanelElems, y, &full[stage]);
-            pa::tma_load_2d(vdst + p * C::kPanelBytes + lane * a.B * 128, &tmV, p * C::kPanelElems, y, &full[stage]);
+          const int off = lane * a.B * D * C::kES;
+          if constexpr (C::kNPanel == 1) {
+            pa::tma_load_2d(kdst + off, &tmK, 0, y, &full[stage]);
+            pa::tma_load_2d(vdst + off, &tmV, 0, y, &full[stage]);
+          } else {
+            pa::tma_load_3d(kdst + off, &tmK, 0, y, 0, &full[stage]);
+            pa::tma_load_3d(vdst + off, &tmV, 0, y, 0, &full[stage]);
           }
         }
         if (tile == 0 && lane == 0) {
@@ -668,6 +856,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     consume_mma<T, D, G, C>(stages, qslots, meta, full, empty, epi, ml, merge, a, warp, lane);
   } else {
   const int grp = lane / L, l = lane % L;
+  const TileAddr ta(a.B, C::kNPanel);
   const int my_tok = token_of_lane<L, R>(l);
   const bool primary = primary_lane<L, R>(l);
   float qf[G][AC];
@@ -735,7 +924,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           for (int k = 0; k < CPL; ++k) {
             const int c = k * L + l;
             const uint4 raw =
-                pa::lds128(ks + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+                pa::lds128(ks + ta.row(row) + ta.chunk(row, c));
             float kv[E];
             ChunkTraits<T>::to_float(raw, kv);
 #pragma unroll
@@ -796,7 +985,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           for (int k = 0; k < CPL; ++k) {
             const int c = k * L + l;
             const uint4 raw =
-                pa::lds128(vs + (c >> 3) * C::kPanelBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+                pa::lds128(vs + ta.row(row) + ta.chunk(row, c));
             float vv[E];
             ChunkTraits<T>::to_float(raw, vv);
 #pragma unroll
@@ -1045,7 +1234,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
-// Tensor map over a cache viewed as [n_blocks*Hk*B rows][d]; box = B rows x 128 bytes.
+// Tensor map over a cache viewed as [n_blocks*Hk*B rows][d].  One box is the B rows of one
+// (block, kv head) with every 128-byte panel of them: with a single panel (d * element size = 128)
+// a 2-D box {128 bytes, B rows}; otherwise a 3-D view {128 bytes, row, panel} whose panel stride
+// (128 bytes) is smaller than its row stride (d * element size), so that the box lands panel by
+// panel ([panel][B rows][128 bytes]), the order the 128-byte swizzle needs for conflict-free
+// ldmatrix.  Every element the view addresses lies inside the cache.
 bool make_cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long long rows, int B) {
   auto enc = get_encoder();
   if (!enc) return false;
@@ -1053,11 +1247,23 @@ bool make_cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long
                                 : dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int es = static_cast<int>(pa::elem_size(dt));
-  cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * es};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(B)};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, t, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  const int panel_elems = 128 / es, n_panel = d / panel_elems;
+  if (n_panel == 1) {
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * es};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(panel_elems), static_cast<cuuint32_t>(B)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, t, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  cuuint64_t gdim[3] = {static_cast<cuuint64_t>(panel_elems), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(n_panel)};
+  cuuint64_t gstride[2] = {static_cast<cuuint64_t>(d) * es, 128};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(panel_elems), static_cast<cuuint32_t>(B),
+                       static_cast<cuuint32_t>(n_panel)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, t, 3, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1211,46 +1417,61 @@ extern "C" pa_status pa_workspace_error(const void* workspace, int* flags, void*
   return pa::ok();
 }
 
-extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
-                               const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
-                               int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq,
-                               int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Everything a decode launch needs, validated: kernel arguments, tensor maps and sizes.
+struct DecodePlan {
+  DecodeArgs a;
+  CUtensorMap tk, tv;
+  WsLayout wl;
+  int g, d, P, max_parts, max_units;
+  pa_dtype kv_dtype, out_dtype;
+};
+
+pa_status prepare_decode(DecodePlan& dp, const char* who, void* out, pa_dtype out_dtype, const void* query,
+                         const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                         const int32_t* context_lens, int S, int H, int Hk, int d, int B, int n_blocks,
+                         int max_blocks_per_seq, int max_context_len, float scale, pa_dtype kv_dtype,
+                         int partition_size, void* workspace, size_t workspace_bytes) {
   if (S < 0 || H <= 0 || Hk <= 0 || n_blocks <= 0 || max_blocks_per_seq < 0 || max_context_len < 0)
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: bad sizes (S=%d H=%d Hk=%d n_blocks=%d)", S, H, Hk, n_blocks);
-  if (H % Hk != 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: H (%d) must be a multiple of Hk (%d)", H, Hk);
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: bad sizes (S=%d H=%d Hk=%d n_blocks=%d)", who, S, H, Hk, n_blocks);
+  if (H % Hk != 0) return pa::fail(PA_ERR_INVALID_ARG, "%s: H (%d) must be a multiple of Hk (%d)", who, H, Hk);
   const int g = H / Hk;
-  if (g != 1 && g != 2 && g != 4 && g != 8) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: H/Hk = %d not in {1,2,4,8}", g);
-  if (d != 64 && d != 128) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: d = %d not in {64,128}", d);
-  if (B != 8 && B != 16 && B != 32) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: B = %d not in {8,16,32}", B);
-  if (!pa::valid_dtype(kv_dtype) || !pa::valid_dtype(out_dtype)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: unknown dtype");
-  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: scale must be finite");
+  if (g != 1 && g != 2 && g != 4 && g != 8) return pa::fail(PA_ERR_UNSUPPORTED, "%s: H/Hk = %d not in {1,2,4,8}", who, g);
+  if (d != 64 && d != 128) return pa::fail(PA_ERR_UNSUPPORTED, "%s: d = %d not in {64,128}", who, d);
+  if (B != 8 && B != 16 && B != 32) return pa::fail(PA_ERR_UNSUPPORTED, "%s: B = %d not in {8,16,32}", who, B);
+  if (!pa::valid_dtype(kv_dtype) || !pa::valid_dtype(out_dtype)) return pa::fail(PA_ERR_INVALID_ARG, "%s: unknown dtype", who);
+  if (!std::isfinite(scale)) return pa::fail(PA_ERR_INVALID_ARG, "%s: scale must be finite", who);
   const int P = partition_size > 0 ? partition_size : default_partition(S, Hk, max_context_len);
-  if (P % kTileTokens != 0 || P > (1 << 24)) return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: partition_size %d must be a positive multiple of 64", P);
+  if (P % kTileTokens != 0 || P > (1 << 24))
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: partition_size %d must be a positive multiple of 64", who, P);
   const int max_parts = max_parts_for(max_context_len, P);
-  if (max_parts > 0xffff) return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: more than 65535 partitions per sequence");
+  if (max_parts > 0xffff) return pa::fail(PA_ERR_UNSUPPORTED, "%s: more than 65535 partitions per sequence", who);
   if (static_cast<long long>(max_blocks_per_seq) * B < max_context_len)
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: max_blocks_per_seq * B < max_context_len");
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: max_blocks_per_seq * B < max_context_len", who);
   const long long rows = static_cast<long long>(n_blocks) * Hk * B;
   if (rows >= (1ll << 31) || static_cast<long long>(S) * Hk * max_parts > (1ll << 31))
-    return pa::fail(PA_ERR_UNSUPPORTED, "pa_decode: problem too large for 32-bit indices");
-  if (S == 0) return pa::ok();
+    return pa::fail(PA_ERR_UNSUPPORTED, "%s: problem too large for 32-bit indices", who);
+  dp.g = g;
+  dp.d = d;
+  dp.P = P;
+  dp.max_parts = max_parts;
+  dp.kv_dtype = kv_dtype;
+  dp.out_dtype = out_dtype;
+  if (S == 0) return PA_OK;
   if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: null pointer");
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: null pointer", who);
   if (!pa::aligned16(out) || !pa::aligned16(query) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: tensors must be 16-byte aligned");
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", who);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: workspace must be 256-byte aligned");
-  const WsLayout wl = ws_layout(S, H, Hk, d, max_parts);
-  if (workspace_bytes < wl.total)
-    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode: workspace of %zu bytes < %zu needed", workspace_bytes, wl.total);
-
-  CUtensorMap tk, tv;
-  if (!make_cache_map(&tk, k_cache, kv_dtype, d, rows, B) || !make_cache_map(&tv, v_cache, kv_dtype, d, rows, B))
-    return pa::fail(PA_ERR_CUDA, "pa_decode: could not encode the cache tensor maps");
-
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+  dp.wl = ws_layout(S, H, Hk, d, max_parts);
+  if (workspace_bytes < dp.wl.total)
+    return pa::fail(PA_ERR_INVALID_ARG, "%s: workspace of %zu bytes < %zu needed", who, workspace_bytes, dp.wl.total);
+  if (!make_cache_map(&dp.tk, k_cache, kv_dtype, d, rows, B) || !make_cache_map(&dp.tv, v_cache, kv_dtype, d, rows, B))
+    return pa::fail(PA_ERR_CUDA, "%s: could not encode the cache tensor maps", who);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  DecodeArgs a;
+  DecodeArgs& a = dp.a;
   a.q = query;
   a.out = out;
   a.out_dtype = out_dtype;
@@ -1265,31 +1486,116 @@ extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query,
   a.P = P;
   a.max_c = max_context_len;
   a.scale_log2 = scale * kLog2e;
-  a.items = reinterpret_cast<const int2*>(ws + wl.items);
+  a.items = reinterpret_cast<const int2*>(ws + dp.wl.items);
   a.hdr = reinterpret_cast<int*>(ws);
-  a.part_o = reinterpret_cast<float*>(ws + wl.part_o);
-  a.part_m = reinterpret_cast<float*>(ws + wl.part_m);
-  a.part_l = reinterpret_cast<float*>(ws + wl.part_l);
+  a.part_o = reinterpret_cast<float*>(ws + dp.wl.part_o);
+  a.part_m = reinterpret_cast<float*>(ws + dp.wl.part_m);
+  a.part_l = reinterpret_cast<float*>(ws + dp.wl.part_l);
   a.max_parts = max_parts;
-
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, context_lens, S, Hk, P,
-                             max_context_len, reinterpret_cast<int2*>(ws + wl.items), a.hdr);
-  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: plan launch failed: %s", cudaGetErrorString(e));
-
   const long long units = static_cast<long long>(S) * Hk * max_parts;
-  const int max_units = static_cast<int>(units < (1ll << 30) ? units : (1ll << 30));
-  if (kv_dtype == PA_F32) e = dispatch_d<float, false>(d, g, tk, tv, a, max_units, st);
-  else if (kv_dtype == PA_F16) e = dispatch_16bit<__half>(d, g, tk, tv, a, max_units, st);
-  else e = dispatch_16bit<__nv_bfloat16>(d, g, tk, tv, a, max_units, st);
-  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s", cudaGetErrorString(e));
+  dp.max_units = static_cast<int>(units < (1ll << 30) ? units : (1ll << 30));
+  return PA_OK;
+}
 
-  if (max_parts > 1) {
-    e = d == 64 ? launch_combine<64>(out, out_dtype, a.part_o, a.part_m, a.part_l, context_lens, S, H, max_parts, P, 2, st)
-                : launch_combine<128>(out, out_dtype, a.part_o, a.part_m, a.part_l, context_lens, S, H, max_parts, P, 2, st);
-    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: combine launch failed: %s", cudaGetErrorString(e));
+// The decode kernel and, for split sequences, the combine; both behind the plan with PDL.
+pa_status launch_decode_and_combine(const DecodePlan& dp, const char* who, cudaStream_t st) {
+  const DecodeArgs& a = dp.a;
+  cudaError_t e;
+  if (dp.kv_dtype == PA_F32) e = dispatch_d<float, false>(dp.d, dp.g, dp.tk, dp.tv, a, dp.max_units, st);
+  else if (dp.kv_dtype == PA_F16) e = dispatch_16bit<__half>(dp.d, dp.g, dp.tk, dp.tv, a, dp.max_units, st);
+  else e = dispatch_16bit<__nv_bfloat16>(dp.d, dp.g, dp.tk, dp.tv, a, dp.max_units, st);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: decode launch failed: %s", who, cudaGetErrorString(e));
+  if (dp.max_parts > 1) {
+    e = dp.d == 64 ? launch_combine<64>(a.out, dp.out_dtype, a.part_o, a.part_m, a.part_l, a.lens, a.S, a.H,
+                                        dp.max_parts, dp.P, 2, st)
+                   : launch_combine<128>(a.out, dp.out_dtype, a.part_o, a.part_m, a.part_l, a.lens, a.S, a.H,
+                                         dp.max_parts, dp.P, 2, st);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: combine launch failed: %s", who, cudaGetErrorString(e));
   }
   return pa::ok();
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                               int S, int H, int Hk, int d, int B, int n_blocks, int max_blocks_per_seq,
+                               int max_context_len, float scale, pa_dtype kv_dtype, int partition_size,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  DecodePlan dp;
+  const pa_status ps = prepare_decode(dp, "pa_decode", out, out_dtype, query, k_cache, v_cache, block_tables,
+                                      context_lens, S, H, Hk, d, B, n_blocks, max_blocks_per_seq, max_context_len,
+                                      scale, kv_dtype, partition_size, workspace, workspace_bytes);
+  if (ps != PA_OK) return ps;
+  if (S == 0) return pa::ok();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, context_lens, S, Hk, dp.P,
+                                   max_context_len, reinterpret_cast<int2*>(const_cast<int2*>(dp.a.items)), dp.a.hdr);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: plan launch failed: %s", cudaGetErrorString(e));
+  return launch_decode_and_combine(dp, "pa_decode", st);
+}
+
+extern "C" pa_status pa_decode_step(void* out, pa_dtype out_dtype, const void* query, void* k_cache, void* v_cache,
+                                    const int32_t* block_tables, const int32_t* context_lens, const void* key,
+                                    const void* value, const int64_t* slot_mapping, int T, const int32_t* pairs,
+                                    const int32_t* n_pairs, int max_pairs, int S, int H, int Hk, int d, int B,
+                                    int n_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                                    pa_dtype kv_dtype, int partition_size, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  DecodePlan dp;
+  const pa_status ps = prepare_decode(dp, "pa_decode_step", out, out_dtype, query, k_cache, v_cache, block_tables,
+                                      context_lens, S, H, Hk, d, B, n_blocks, max_blocks_per_seq, max_context_len,
+                                      scale, kv_dtype, partition_size, workspace, workspace_bytes);
+  if (ps != PA_OK) return ps;
+  if (T < 0 || max_pairs < 0 || max_pairs > kMaxStepPairs)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_step: need T >= 0 and 0 <= max_pairs <= %d (T=%d, max_pairs=%d)",
+                    kMaxStepPairs, T, max_pairs);
+  if ((T > 0 && (!key || !value || !slot_mapping)) || (max_pairs > 0 && !pairs) || !k_cache || !v_cache)
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_step: null pointer");
+  if (!pa::aligned16(k_cache) || !pa::aligned16(v_cache) || (T > 0 && (!pa::aligned16(key) || !pa::aligned16(value))))
+    return pa::fail(PA_ERR_INVALID_ARG, "pa_decode_step: caches, key and value must be 16-byte aligned");
+  const int es = static_cast<int>(pa::elem_size(kv_dtype));
+  PrologueArgs w;
+  w.kc = static_cast<uint4*>(k_cache);
+  w.vc = static_cast<uint4*>(v_cache);
+  w.key = static_cast<const uint4*>(key);
+  w.value = static_cast<const uint4*>(value);
+  w.slots = slot_mapping;
+  w.pairs = pairs;
+  w.n_pairs_dev = n_pairs;
+  w.T = T;
+  w.max_pairs = max_pairs;
+  w.Hk = Hk;
+  w.chunks = d * es / 16;
+  w.B = B;
+  w.n_blocks = n_blocks;
+  w.vec_per_block = static_cast<long long>(Hk) * B * d * es / 16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (S == 0) {
+    // nothing to decode: the copies and writes alone, in their order
+    pa_status s2 = max_pairs > 0 ? (n_pairs ? pa::copy_blocks_counted(k_cache, v_cache, pairs, n_pairs, max_pairs, Hk,
+                                                                       d, B, n_blocks, kv_dtype, stream)
+                                            : pa_copy_blocks(k_cache, v_cache, pairs, max_pairs, Hk, d, B, n_blocks,
+                                                             kv_dtype, stream))
+                                 : PA_OK;
+    if (s2 == PA_OK) s2 = pa_cache_write(k_cache, v_cache, key, value, slot_mapping, T, Hk, d, B, n_blocks, kv_dtype, stream);
+    return s2;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // one CTA for the plan, then workers: one per pair (the count on the device may be smaller) and
+  // enough warps for the tokens, at most four per SM
+  long long workers = max_pairs;
+  const long long for_tokens = (static_cast<long long>(T) + kPrologueThreads / 32 - 1) / (kPrologueThreads / 32);
+  if (workers < for_tokens) workers = for_tokens;
+  if (workers > 4LL * sms) workers = 4LL * sms;
+  if (workers < 1) workers = 1;
+  cudaError_t e = launch_pdl(step_prologue_kernel, dim3(static_cast<unsigned>(1 + workers)), dim3(kPrologueThreads), 0,
+                             st, w, context_lens, S, Hk, dp.P, max_context_len,
+                             reinterpret_cast<int2*>(const_cast<int2*>(dp.a.items)), dp.a.hdr);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode_step: prologue launch failed: %s", cudaGetErrorString(e));
+  return launch_decode_and_combine(dp, "pa_decode_step", st);
 }
 
 extern "C" pa_status pa_combine(void* out, pa_dtype out_dtype, const float* part_o, const float* part_m,
@@ -1313,8 +1619,12 @@ extern "C" pa_status pa_combine(void* out, pa_dtype out_dtype, const float* part
 // ---- decode without any device allocation --------------------------------------------------------
 // The decode workspace of pa_decode_noalloc lives in this file-scope device array instead of
 // caller memory.  Every GPU that loads the library holds it until the process exits.  In host
-// code `g_noalloc_scratch` only names a host-side stand-in, so its device address is fetched once
-// per device with cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// code `g_noalloc_scratch` only names a host-side stand-in, so its device address is fetched with
+// cudaGetSymbolAddress (with the device current) and passed to the kernels.  The address belongs
+// to the device's current context: it is looked up once per device and looked up again when that
+// context has changed (a device reset destroys the context, and the module holding the array is
+// loaded again, possibly elsewhere, in the next one).  Contexts are told apart by the driver's
+// context id, which is never reused within a process.
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
@@ -1322,7 +1632,34 @@ __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoAllocSlot {
+  void* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+NoAllocSlot g_noalloc[kMaxDevices];
+
+// Id of the calling thread's current context (0 if it cannot be had, which forces a lookup).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 cudaError_t noalloc_scratch(void** ptr) {
   int dev = 0;
@@ -1330,13 +1667,16 @@ cudaError_t noalloc_scratch(void** ptr) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  NoAllocSlot& slot = g_noalloc[dev];
+  const unsigned long long ctx_id = current_context_id();  // 0 before the runtime has made one current
+  if (!slot.ptr || ctx_id == 0 || slot.ctx_id != ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's context current if needed
     if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_context_id();
   }
-  *ptr = g_noalloc_ptr[dev];
+  *ptr = slot.ptr;
   return cudaSuccess;
 }
 

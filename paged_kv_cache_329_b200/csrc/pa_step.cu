@@ -86,17 +86,26 @@ std::vector<Copy> input_copies(const pa_step_desc& d) {
   return merged;
 }
 
-// copy-on-write copies, cache write, decode
+// copy-on-write copies, cache write, decode (pa_decode_step: the copies, the writes and the plan in
+// one kernel, the pair count read on the device)
 pa_status record_kernels(const pa_step_desc& d, cudaStream_t s) {
-  pa_status st = pa::copy_blocks_counted(d.k_cache, d.v_cache, d.d_pairs, d.d_pairs + 2 * static_cast<size_t>(d.max_pairs),
-                                         d.max_pairs, d.Hk, d.d, d.B, d.n_blocks, d.kv_dtype, s);
-  if (st != PA_OK) return st;
-  st = pa_cache_write(d.k_cache, d.v_cache, d.d_key, d.d_value, d.d_slots, d.S, d.Hk, d.d, d.B, d.n_blocks, d.kv_dtype, s);
-  if (st != PA_OK) return st;
-  st = pa_decode(d.d_out, d.out_dtype, d.d_query, d.k_cache, d.v_cache, d.d_tables, d.d_lens, d.S, d.H, d.Hk, d.d, d.B,
-                 d.n_blocks, d.max_blocks_per_seq, d.max_context_len, d.scale, d.kv_dtype, d.partition_size,
-                 d.workspace, d.workspace_bytes, s);
-  return st;
+  if (d.max_pairs > pa::kMaxStepPairs) {  // too many pairs for the fused form: three calls in order
+    pa_status st = pa::copy_blocks_counted(d.k_cache, d.v_cache, d.d_pairs,
+                                           d.d_pairs + 2 * static_cast<size_t>(d.max_pairs), d.max_pairs, d.Hk, d.d,
+                                           d.B, d.n_blocks, d.kv_dtype, s);
+    if (st == PA_OK)
+      st = pa_cache_write(d.k_cache, d.v_cache, d.d_key, d.d_value, d.d_slots, d.S, d.Hk, d.d, d.B, d.n_blocks,
+                          d.kv_dtype, s);
+    if (st == PA_OK)
+      st = pa_decode(d.d_out, d.out_dtype, d.d_query, d.k_cache, d.v_cache, d.d_tables, d.d_lens, d.S, d.H, d.Hk,
+                     d.d, d.B, d.n_blocks, d.max_blocks_per_seq, d.max_context_len, d.scale, d.kv_dtype,
+                     d.partition_size, d.workspace, d.workspace_bytes, s);
+    return st;
+  }
+  return pa_decode_step(d.d_out, d.out_dtype, d.d_query, d.k_cache, d.v_cache, d.d_tables, d.d_lens, d.d_key,
+                        d.d_value, d.d_slots, d.S, d.d_pairs, d.d_pairs + 2 * static_cast<size_t>(d.max_pairs),
+                        d.max_pairs, d.S, d.H, d.Hk, d.d, d.B, d.n_blocks, d.max_blocks_per_seq, d.max_context_len,
+                        d.scale, d.kv_dtype, d.partition_size, d.workspace, d.workspace_bytes, s);
 }
 
 size_t out_bytes(const pa_step_desc& d) {

@@ -268,6 +268,90 @@ def test_copy_blocks_bit_exact(oracle_mod, dtype):
     assert torch.equal(vd.cpu().view(bits), v_ref.view(bits))
 
 
+# ---- the fused decode step (pa_decode_step) -----------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,B,d,g", [(torch.bfloat16, 16, 128, 4), (torch.float16, 8, 128, 1),
+                                         (torch.float32, 32, 64, 2), (torch.bfloat16, 8, 64, 8)])
+def test_decode_step_matches_copy_write_decode(oracle_mod, dtype, B, d, g):
+    # Sequences forked from shared parents reserve 1-3 new tokens each (copy-on-write pairs where a
+    # shared last block has room), plus padding tokens (slot -1).  The block manager is the
+    # oracle's model; pa_decode_step must equal copy -> write -> decode by the oracle, with the
+    # pair count read on the device and garbage rows past it ignored.
+    from oracle.allocator import BlockManagerModel
+
+    Hk, n_blocks = 2, 600
+    H = g * Hk
+    mgr = BlockManagerModel(n_blocks, B)
+    rnd = torch.Generator().manual_seed(800 + B + d)
+    roots = []
+    for i in range(6):
+        r = mgr.seq_create()
+        mgr.reserve_slots(r, int(torch.randint(1, 300, (1,), generator=rnd)))
+        roots.append(r)
+    seqs = []
+    for r in roots:
+        seqs += [r] + [mgr.seq_fork(r) for _ in range(int(torch.randint(0, 4, (1,), generator=rnd)))]
+    slots, pairs = [], []
+    for s_ in seqs:
+        n_new = int(torch.randint(1, 4, (1,), generator=rnd))
+        sl, pr = mgr.reserve_slots(s_, n_new)
+        slots += sl + ([-1] if n_new == 2 else [])
+        pairs += pr
+    assert len(pairs) > 0
+    tables, lens = mgr.build_block_tables(seqs, max(len(mgr.seq_table(x)) for x in seqs))
+    tables, lens = torch.tensor(tables, dtype=torch.int32), torch.tensor(lens, dtype=torch.int32)
+    slots = torch.tensor(slots, dtype=torch.int64)
+    T, S = slots.numel(), len(seqs)
+    g_in = W.generator(801 + B)
+    kc = W.randn(g_in, (n_blocks, Hk, B, d), dtype)
+    vc = W.randn(g_in, (n_blocks, Hk, B, d), dtype)
+    key = W.randn(g_in, (T, Hk, d), dtype)
+    val = W.randn(g_in, (T, Hk, d), dtype)
+    q = W.randn(g_in, (S, H, d), dtype)
+    pr = torch.tensor(pairs, dtype=torch.int32).reshape(-1, 2)
+    # rows past the count: copies that would overwrite live blocks if they were made
+    assert int(tables[0, 0]) != int(tables[-1, 0])
+    padded = torch.cat([pr, torch.tensor([[int(tables[0, 0]), int(tables[-1, 0])]] * 5, dtype=torch.int32)])
+    n_dev = torch.tensor([pr.shape[0]], dtype=torch.int32, device="cuda")
+    k_ref, v_ref = oracle_mod.copy_blocks(kc, vc, pr)
+    k_ref, v_ref = oracle_mod.cache_write(k_ref, v_ref, key, val, slots)
+    ref = oracle_mod.decode(q, k_ref, v_ref, tables, lens, 1.0 / math.sqrt(d))
+    kd, vd = kc.cuda(), vc.cuda()
+    max_c = int(lens.max())
+    for P in (0, 64):
+        kd.copy_(kc.cuda())
+        vd.copy_(vc.cuda())
+        ws = api.alloc_workspace(S, H, Hk, d, max_c, P)
+        out = api.pa_decode_step(q.cuda(), kd, vd, tables.cuda(), lens.cuda(), key.cuda(), val.cuda(), slots.cuda(),
+                                 padded.cuda(), n_pairs=n_dev, max_context_len=max_c, out_dtype=torch.float32,
+                                 partition_size=P, workspace=ws)
+        torch.cuda.synchronize()
+        assert api.workspace_error(ws) == 0
+        bits = torch.int32 if dtype == torch.float32 else torch.int16
+        assert torch.equal(kd.cpu().view(bits), k_ref.view(bits)), f"K cache P={P}"
+        assert torch.equal(vd.cpu().view(bits), v_ref.view(bits)), f"V cache P={P}"
+        _assert_close(out.cpu(), ref, dtype, f"decode step {dtype} B={B} d={d} g={g} P={P}")
+    # the pair count given on the host instead (no device count): the same result
+    kd.copy_(kc.cuda())
+    vd.copy_(vc.cuda())
+    out = api.pa_decode_step(q.cuda(), kd, vd, tables.cuda(), lens.cuda(), key.cuda(), val.cuda(), slots.cuda(),
+                             pr.cuda(), max_context_len=max_c, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _assert_close(out.cpu(), ref, dtype, "decode step, host count")
+
+
+def test_decode_step_without_pairs_or_tokens(oracle_mod):
+    case = W.paged_case("step0", [5, 300, 0, 64], 8, 2, 128, 16, torch.bfloat16, 810)
+    dev = case.to("cuda")
+    none_i32 = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    key = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    slots = torch.empty((0,), dtype=torch.int64, device="cuda")
+    out = api.pa_decode_step(dev.q, dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens, key, key, slots,
+                             none_i32, max_context_len=300, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _assert_close(out.cpu(), _oracle(oracle_mod, case), torch.bfloat16, "step without pairs or tokens")
+
+
 # ---- the captured step (pa_step_*) ------------------------------------------------------------------
 
 def test_captured_step_matches_separate_calls(oracle_mod):
