@@ -23,8 +23,9 @@ struct pa_alloc {
   int B = 0;
   std::vector<int32_t> ref;   // reference count per physical block (0 = free)
   std::vector<int32_t> free;  // LIFO stack of free ids; back() is handed out next
-  std::unordered_map<int32_t, Seq> seqs;
-  std::vector<std::vector<int32_t>> spare;  // table storage of freed sequences, reused by new ones
+  using SeqMap = std::unordered_map<int32_t, Seq>;
+  SeqMap seqs;
+  std::vector<SeqMap::node_type> spare;  // freed sequences' map nodes (with their table storage)
   int32_t next_seq = 0;
 };
 
@@ -43,15 +44,19 @@ void release(pa_alloc* a, int32_t b) {  // caller checked allocated(a, b)
   if (--a->ref[b] == 0) a->free.push_back(b);
 }
 
-// An empty table for a new sequence, taken from freed sequences' storage when there is some (a
-// serving loop forks and frees a batch of sequences every step; this keeps that free of
-// allocations once the pool has warmed up).
-std::vector<int32_t> fresh_table(pa_alloc* a) {
-  if (a->spare.empty()) return {};
-  std::vector<int32_t> t = std::move(a->spare.back());
+// Inserts a new sequence `id` with an empty table and returns it.  The map node and the table
+// storage of a freed sequence are reused when there is one: a serving loop forks and frees a batch
+// of sequences every step, and once as many sequences have been freed as are created per step, a
+// step allocates neither nodes nor tables (the map's bucket array grows only when the number of
+// live sequences exceeds every earlier count).
+pa_alloc::Seq& insert_seq(pa_alloc* a, int32_t id) {
+  if (a->spare.empty()) return a->seqs.emplace(id, pa_alloc::Seq{}).first->second;
+  pa_alloc::SeqMap::node_type node = std::move(a->spare.back());
   a->spare.pop_back();
-  t.clear();
-  return t;
+  node.key() = id;
+  node.mapped().table.clear();
+  node.mapped().n_tokens = 0;
+  return a->seqs.insert(std::move(node)).position->second;
 }
 
 }  // namespace
@@ -109,9 +114,7 @@ int pa_alloc_num_free(const pa_alloc* a) { return a ? static_cast<int>(a->free.s
 pa_status pa_seq_create(pa_alloc* a, int32_t* seq_id) {
   if (!a || !seq_id) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_create: null argument");
   const int32_t id = a->next_seq++;
-  pa_alloc::Seq s;
-  s.table = fresh_table(a);
-  a->seqs.emplace(id, std::move(s));
+  insert_seq(a, id);
   *seq_id = id;
   return pa::ok();
 }
@@ -120,13 +123,13 @@ pa_status pa_seq_fork(pa_alloc* a, int32_t parent, int32_t* child) {
   if (!a || !child) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_fork: null argument");
   auto it = a->seqs.find(parent);
   if (it == a->seqs.end()) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_fork: unknown sequence %d", parent);
-  pa_alloc::Seq copy;
-  copy.table = fresh_table(a);
-  copy.table.assign(it->second.table.begin(), it->second.table.end());
-  copy.n_tokens = it->second.n_tokens;
-  for (int32_t b : copy.table) ++a->ref[b];
   const int32_t id = a->next_seq++;
-  a->seqs.emplace(id, std::move(copy));
+  // the parent's entry stays valid: unordered_map references survive insertion (rehash included)
+  const pa_alloc::Seq& parent_seq = it->second;
+  pa_alloc::Seq& s = insert_seq(a, id);
+  s.table.assign(parent_seq.table.begin(), parent_seq.table.end());
+  s.n_tokens = parent_seq.n_tokens;
+  for (int32_t b : s.table) ++a->ref[b];
   *child = id;
   return pa::ok();
 }
@@ -136,8 +139,8 @@ pa_status pa_seq_free(pa_alloc* a, int32_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return pa::fail(PA_ERR_INVALID_ARG, "pa_seq_free: unknown sequence %d", seq_id);
   for (int32_t b : it->second.table) release(a, b);
-  if (a->spare.size() < 4096) a->spare.push_back(std::move(it->second.table));
-  a->seqs.erase(it);
+  if (a->spare.size() < 4096) a->spare.push_back(a->seqs.extract(it));
+  else a->seqs.erase(it);
   return pa::ok();
 }
 
