@@ -454,13 +454,22 @@ def run_pa(args, rank, world, local_rank):
         e2e_bytes += (c_sum * Hk * d * 2 * es + S * H * d * es * 2 + 4 * nb_sum + 4 * S
                       + 2 * (S * Hk * d * es * 2) + 8 * S + pr.shape[0] * 2 * (Hk * B * d * es) * 2)
 
+    host_busy = {"prepare": [], "launch": [], "wait": []}   # host seconds per step, by phase
+
     def e2e_run(n):
         for i in range(n):
             st = steps[i % E2E_DEPTH]
+            t0 = time.perf_counter()
             if i >= E2E_DEPTH:
                 st.wait()                # step i-E2E_DEPTH's output is in st.h_out; its buffers are free
+            t1 = time.perf_counter()
             prepare(st)                  # overlaps the GPU running the previous steps
+            t2 = time.perf_counter()
             st.launch_async(stream)
+            t3 = time.perf_counter()
+            host_busy["wait"].append(t1 - t0)
+            host_busy["prepare"].append(t2 - t1)
+            host_busy["launch"].append(t3 - t2)
         for st in steps[:min(n, E2E_DEPTH)]:
             st.wait()
         stream.synchronize()
@@ -468,6 +477,8 @@ def run_pa(args, rank, world, local_rank):
     e2e_run(2)  # warm-up (also grows every sequence by two tokens)
     e2e_bytes = 0
     host_s.clear()
+    for v in host_busy.values():
+        v.clear()
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -558,6 +569,7 @@ def run_pa(args, rank, world, local_rank):
             "steps": e2e_steps,
             "ms_per_step": round(e2e_ms / e2e_steps, 5),
             "host_block_manager_ms": round(1e3 * statistics.median(host_s), 5) if host_s else None,
+            "host_ms_per_step": {k: round(1e3 * statistics.mean(v), 5) for k, v in host_busy.items() if v},
             "note": "per step: host block manager (prepared while the GPU runs the previous step), H2D "
                     "of the step's inputs from pinned memory, one replay of the captured kernels "
                     "(pa_decode_step: copies, writes and plan, decode, combine), D2H of o; the copies run on "
@@ -765,10 +777,10 @@ def run_cache_ops(args, rank, world, local_rank):
     """The copy-on-write copy and the slot-mapped write at sizes where they are bandwidth-bound:
     4096 (src, dst) pairs of gqa8k-shaped blocks (8 kv heads x 16 tokens x 128 dims, bf16; 256 MiB
     written, twice the L2, so the copies' writes reach DRAM within the launch) and 65536 new tokens
-    written through a random slot mapping into a 65536-block pool."""
+    written through a random slot mapping into a 16384-block pool (1 GiB of K and V)."""
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    n_blocks, Hk, B, d, dt = 65536, 8, 16, 128, torch.bfloat16
+    n_blocks, Hk, B, d, dt = 16384, 8, 16, 128, torch.bfloat16
     gen = torch.Generator(device=dev).manual_seed(31 + rank)
     kc = torch.randn((n_blocks, Hk, B, d), generator=gen, device=dev).to(dt)
     vc = torch.randn((n_blocks, Hk, B, d), generator=gen, device=dev).to(dt)

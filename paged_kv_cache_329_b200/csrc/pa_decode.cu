@@ -119,14 +119,20 @@ __device__ __forceinline__ int tile_bucket(int ntok, int P) {
 
 constexpr int kPlanCache = 4096;  // lengths kept in shared memory between the two passes
 
+constexpr int kPlanLong = 1024;   // sequences whose whole-partition items a warp writes
+
 struct PlanSmem {
   int count[kBuckets], cursor[kBuckets];
   int c_cache[kPlanCache];
+  int2 long_seq[kPlanLong];
+  int n_long;
 };
 
 // Lists the units of one decode launch into items[] and resets the workspace header; run by one
 // whole CTA (any block size that is a multiple of 32).  Each bucket's start is an exclusive
-// prefix sum over the buckets from the longest down, taken by the first warp.
+// prefix sum over the buckets from the longest down, taken by the first warp; a thread per
+// sequence then writes its items, except that a warp writes the whole-partition items of a
+// sequence that has more than 32 of them.
 __device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restrict__ lens, int S, int Hk, int P,
                                            int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -172,16 +178,36 @@ __device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restri
       hdr[kHdrNumItems] = incl;
     }
   }
+  if (tid == 0) sm.n_long = 0;
   __syncthreads();
+  // A thread per sequence takes its places and writes its last-partition items; a sequence with
+  // more than 32 whole-partition items leaves those to a warp (below).
   for (int s = tid; s < S; s += nt) {
     const int c = s < kPlanCache ? sm.c_cache[s] : min(max(lens[s], 0), max_c);
     const int f = max(1, (c + P - 1) / P) - 1;
     if (f > 0) {
       const int base = atomicAdd(&sm.cursor[nb - 1], f * Hk);
-      for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+      if (f * Hk <= 32 || s >= kPlanCache) {
+        for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+      } else {
+        const int k = atomicAdd(&sm.n_long, 1);
+        if (k < kPlanLong) {
+          sm.long_seq[k] = make_int2(s, base);
+        } else {  // more long sequences than the list holds: this thread writes them itself
+          atomicSub(&sm.n_long, 1);
+          for (int i = 0; i < f * Hk; ++i) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
+        }
+      }
     }
     const int base = atomicAdd(&sm.cursor[tile_bucket(c - f * P, P)], Hk);
     for (int kh = 0; kh < Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | f);
+  }
+  __syncthreads();
+  const int lane = tid & 31;
+  for (int k = tid >> 5; k < sm.n_long; k += nt >> 5) {
+    const int s = sm.long_seq[k].x, base = sm.long_seq[k].y;
+    const int f = max(1, (sm.c_cache[s] + P - 1) / P) - 1;
+    for (int i = lane; i < f * Hk; i += 32) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
   }
   const int any_clamped = __syncthreads_or(clamped);
   if (tid == 0) hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
@@ -1146,72 +1172,98 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 }
 
 // ---- log-sum-exp combine -----------------------------------------------------------------------
-// One warp per (sequence, query head); lane owns D/32 consecutive dims.  Sequences with fewer
-// than min_parts partitions are skipped (the decode kernel already wrote them).
-template <class OutT, int D>
-__global__ void __launch_bounds__(256) combine_kernel(OutT* __restrict__ out, const float* __restrict__ part_o,
-                                                      const float* __restrict__ part_m,
-                                                      const float* __restrict__ part_l,
-                                                      const int32_t* __restrict__ lens, int S, int H,
-                                                      int max_parts, int P, int min_parts) {
+// WPR warps per (sequence, query head); lane owns D/32 consecutive dims.  With WPR > 1 the warps of
+// a row take interleaved batches of 32 partitions (batch b to warp b % WPR) and their sums are
+// added in a fixed order through shared memory, so that rows with many partitions keep more loads
+// in flight.  Sequences with fewer than min_parts partitions are skipped (the decode kernel
+// already wrote them).
+constexpr int kCombineThreads = 256;
+
+template <class OutT, int D, int WPR>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(OutT* __restrict__ out, const float* __restrict__ part_o,
+                                                                  const float* __restrict__ part_m,
+                                                                  const float* __restrict__ part_l,
+                                                                  const int32_t* __restrict__ lens, int S, int H,
+                                                                  int max_parts, int P, int min_parts) {
   // Partitions past max_parts are never read: a length that needs more is cut to max_parts * P.
   pa::grid_dependency_wait();  // launched right behind the decode grid: its partials must be complete
   constexpr int PER = D / 32;
-  const long long gw = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= static_cast<long long>(S) * H) return;
-  const int s = static_cast<int>(gw / H);
-  const int c = max(lens[s], 0);
-  const int np = min((c + P - 1) / P, max_parts);
-  OutT* o = out + gw * D + lane * PER;
-  float res[PER];
-  if (np == 0) {  // empty context: zeros (the decode kernel already wrote them when min_parts > 1)
-    if (min_parts <= 1) {
-#pragma unroll
-      for (int e = 0; e < PER; ++e) res[e] = 0.f;
-      pa::store_pairs<OutT, PER>(o, res);
-    }
-    return;
-  }
-  if (np < min_parts) return;
-  const float* pm = part_m + gw * max_parts;
-  const float* pl = part_l + gw * max_parts;
-  float mx = -INFINITY;
-  for (int p = lane; p < np; p += 32) mx = fmaxf(mx, pm[p]);
-#pragma unroll
-  for (int msk = 16; msk >= 1; msk >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+  constexpr int kRowsPerCta = kCombineThreads / 32 / WPR;
+  __shared__ float red_acc[WPR > 1 ? kRowsPerCta * (WPR - 1) * D : 1];
+  __shared__ float red_den[WPR > 1 ? kRowsPerCta * (WPR - 1) : 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_in_cta = warp / WPR, sub = warp % WPR;
+  const long long gw = static_cast<long long>(blockIdx.x) * kRowsPerCta + row_in_cta;
+  bool write = false;  // this row's output is written here (by sub-warp 0)
+  int np = 0;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float den = 0.f;
-  if (mx != -INFINITY) {
-    // 32 partitions at a time: lane j computes partition (base + j)'s weight, then every lane
-    // accumulates its dims over the 32 with independent loads in flight.
-    for (int base = 0; base < np; base += 32) {
-      const int p = base + lane;
-      float w = 0.f;
-      if (p < np) {
-        const float mp = pm[p];
-        w = mp == -INFINITY ? 0.f : expf(mp - mx);
-        den = fmaf(w, pl[p], den);
-      }
-      const int cnt = min(32, np - base);
-      const float* src = part_o + (gw * max_parts + base) * D + lane * PER;
-#pragma unroll 8
-      for (int j = 0; j < cnt; ++j) {
-        const float wj = __shfl_sync(0xffffffffu, w, j);
+  if (gw < static_cast<long long>(S) * H) {
+    const int s = static_cast<int>(gw / H);
+    const int c = max(lens[s], 0);
+    np = min((c + P - 1) / P, max_parts);
+    // empty context: zeros (the decode kernel already wrote them when min_parts > 1)
+    write = np == 0 ? min_parts <= 1 : np >= min_parts;
+  }
+  if (write && np > 0) {
+    const float* pm = part_m + gw * max_parts;
+    const float* pl = part_l + gw * max_parts;
+    float mx = -INFINITY;
+    for (int p = lane; p < np; p += 32) mx = fmaxf(mx, pm[p]);
 #pragma unroll
-        for (int e = 0; e < PER; e += 2) {
-          const float2 v = *reinterpret_cast<const float2*>(src + static_cast<size_t>(j) * D + e);
-          acc[e] = fmaf(wj, v.x, acc[e]);
-          acc[e + 1] = fmaf(wj, v.y, acc[e + 1]);
+    for (int msk = 16; msk >= 1; msk >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+    if (mx != -INFINITY) {
+      // 32 partitions at a time: lane j computes partition (base + j)'s weight, then every lane
+      // accumulates its dims over the 32 with independent loads in flight.
+      for (int base = sub * 32; base < np; base += 32 * WPR) {
+        const int p = base + lane;
+        float w = 0.f;
+        if (p < np) {
+          const float mp = pm[p];
+          w = mp == -INFINITY ? 0.f : expf(mp - mx);
+          den = fmaf(w, pl[p], den);
+        }
+        const int cnt = min(32, np - base);
+        const float* src = part_o + (gw * max_parts + base) * D + lane * PER;
+#pragma unroll 8
+        for (int j = 0; j < cnt; ++j) {
+          const float wj = __shfl_sync(0xffffffffu, w, j);
+#pragma unroll
+          for (int e = 0; e < PER; e += 2) {
+            const float2 v = *reinterpret_cast<const float2*>(src + static_cast<size_t>(j) * D + e);
+            acc[e] = fmaf(wj, v.x, acc[e]);
+            acc[e + 1] = fmaf(wj, v.y, acc[e + 1]);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int msk = 16; msk >= 1; msk >>= 1) den += __shfl_xor_sync(0xffffffffu, den, msk);
+      for (int msk = 16; msk >= 1; msk >>= 1) den += __shfl_xor_sync(0xffffffffu, den, msk);
+    }
   }
+  if constexpr (WPR > 1) {
+    // sub-warps 1 .. WPR-1 hand their sums to sub-warp 0, which adds them in index order
+    if (sub > 0) {
+      float* dst = red_acc + (row_in_cta * (WPR - 1) + sub - 1) * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) dst[e] = acc[e];
+      if (lane == 0) red_den[row_in_cta * (WPR - 1) + sub - 1] = den;
+    }
+    __syncthreads();
+    if (sub > 0) return;
+#pragma unroll
+    for (int k = 0; k < WPR - 1; ++k) {
+      const float* src = red_acc + (row_in_cta * (WPR - 1) + k) * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] += src[e];
+      den += red_den[row_in_cta * (WPR - 1) + k];
+    }
+  }
+  if (!write) return;
+  OutT* o = out + gw * D + lane * PER;
   const float inv = den > 0.f ? 1.f / den : 0.f;
+  float res[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) res[e] = acc[e] * inv;
   pa::store_pairs<OutT, PER>(o, res);
@@ -1285,21 +1337,30 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+template <int D, int WPR>
+cudaError_t launch_combine_w(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
+                             const int32_t* lens, int S, int H, int max_parts, int P, int min_parts, cudaStream_t st) {
+  constexpr int kRowsPerCta = kCombineThreads / 32 / WPR;
+  const long long rows = static_cast<long long>(S) * H;
+  const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta)), block(kCombineThreads);
+  if (grid.x == 0) return cudaSuccess;
+  if (out_dtype == PA_F32)
+    return launch_pdl(combine_kernel<float, D, WPR>, grid, block, 0, st, static_cast<float*>(out), po, pm, pl, lens, S,
+                      H, max_parts, P, min_parts);
+  if (out_dtype == PA_F16)
+    return launch_pdl(combine_kernel<__half, D, WPR>, grid, block, 0, st, static_cast<__half*>(out), po, pm, pl, lens,
+                      S, H, max_parts, P, min_parts);
+  return launch_pdl(combine_kernel<__nv_bfloat16, D, WPR>, grid, block, 0, st, static_cast<__nv_bfloat16*>(out), po,
+                    pm, pl, lens, S, H, max_parts, P, min_parts);
+}
+
+// Rows with many partitions (more than two batches of 32) get four warps each.
 template <int D>
 cudaError_t launch_combine(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
                            const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
                            cudaStream_t st) {
-  const long long threads = static_cast<long long>(S) * H * 32;
-  const dim3 grid(static_cast<unsigned>((threads + 255) / 256)), block(256);
-  if (grid.x == 0) return cudaSuccess;
-  if (out_dtype == PA_F32)
-    return launch_pdl(combine_kernel<float, D>, grid, block, 0, st, static_cast<float*>(out), po, pm, pl, lens, S, H,
-                      max_parts, P, min_parts);
-  if (out_dtype == PA_F16)
-    return launch_pdl(combine_kernel<__half, D>, grid, block, 0, st, static_cast<__half*>(out), po, pm, pl, lens, S,
-                      H, max_parts, P, min_parts);
-  return launch_pdl(combine_kernel<__nv_bfloat16, D>, grid, block, 0, st, static_cast<__nv_bfloat16*>(out), po, pm,
-                    pl, lens, S, H, max_parts, P, min_parts);
+  return max_parts > 64 ? launch_combine_w<D, 4>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, st)
+                        : launch_combine_w<D, 1>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, st);
 }
 
 struct DeviceInfo {

@@ -463,10 +463,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 // ---- tcgen05 consumers -------------------------------------------------------------------------------
 // 256 query rows per unit in two 128-row halves A and B (one TMEM lane per row in each half).
 // Warps 0-3 own the rows of half A, warps 4-7 those of half B (softmax, P, output); warp 8 is the
-// TMA producer; one lane of warp 9 issues the MMAs of half A, one lane of warp 10 those of half B
-// (a single thread issues one tcgen05.mma about every 100 cycles whatever its size, so one issuer
-// per half doubles the rate at which these small MMAs reach the tensor core); warp 9 also
-// allocates TMEM.  Per 64-key tile j and half h:
+// TMA producer; one lane each of warps 9 and 10 issues the S MMAs of halves A and B, one lane each
+// of warps 11 and 12 their P.V MMAs.  A single thread issues one tcgen05.mma about every 126-134
+// cycles with A in shared memory and 166-186 with A in tensor memory, whatever its N up to 128
+// (measured on B200), and separate issuing warps add up: four issuers keep up with the tensor core
+// where one per half (about 2400 issue cycles per 64-key tile) did not.  Warp 9 also allocates TMEM.
+// Per 64-key tile j and half h:
 //   S_h[128 x 64]  = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
 //   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) back to TMEM
 //   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    A = P_h from TMEM, B = V tile (MN-major: d contiguous)
@@ -477,8 +479,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 constexpr int kURows = 128;                  // rows per half (TMEM lanes)
 constexpr int kUHalves = 2;
 constexpr int kUUnitRows = kURows * kUHalves;
-constexpr int kUProducer = 8, kUMma = 9;    // MMA issuers: warps kUMma (half A) and kUMma + 1 (half B)
-constexpr int kUThreads = 11 * 32;
+constexpr int kUProducer = 8;
+constexpr int kUMmaS = 9;                    // S issuers: warps 9 (half A) and 10 (half B)
+constexpr int kUMmaPV = 11;                  // P.V issuers: warps 11 (half A) and 12 (half B)
+constexpr int kUThreads = 16 * 32;          // four warpgroups: rows (2), producer + issuers, issuer + idle
+// Registers: the CTA launches with 512 x 128.  The row warpgroups raise theirs to kRegsRows and the
+// two others lower theirs to kRegsOther; 2 x 128 x (kRegsRows + kRegsOther) must not exceed
+// 512 x 128, or the raise would wait for registers that are never released.
+constexpr uint32_t kRegsRows = 200, kRegsOther = 56;
+static_assert(2 * 128 * (kRegsRows + kRegsOther) <= 512 * 128, "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;          // S_A 0..63, S_B 64..127, O_A 128.., O_B 128+d.., P_A 384.., P_B 448..
 constexpr uint32_t kTmemP = 384;             // P_h: 32 columns of packed hi pairs, then 32 of lo pairs
 
@@ -527,7 +536,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       pa::mbar_init(&full[i], 1);
-      pa::mbar_init(&empty[i], kUHalves);  // one tcgen05.commit per tile from each half's issuer
+      pa::mbar_init(&empty[i], 2 * kUHalves);  // one tcgen05.commit per tile from each of the 4 issuers
     }
     for (int h = 0; h < kUHalves; ++h) {
       pa::mbar_init(&q_ready[h], kURows);
@@ -539,7 +548,7 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
     pa::mbar_init(teardown, kUUnitRows);
     pa::fence_barrier_init();
   }
-  if (warp == kUMma) {
+  if (warp == kUMmaS) {
     pa::tmem_alloc(tmem_slot, kTmemCols);
     pa::tmem_relinquish();
   }
@@ -548,103 +557,124 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   pa::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pa::grid_dependency_wait();
+  if (warp >= 8) {
+    // every path of warps 8-15 ends in a return below: the row code after this block runs with the
+    // raised budget only
+    pa::setmaxnreg_dec<kRegsOther>();
+    if (warp > kUMmaPV + 1) return;  // warps 13-15 only complete the last warpgroup
 
-  if (warp == kUProducer) {
-    produce_units<D, C>(smem, meta, full, empty, tmK, tmV, a, lane);
-    return;
-  }
+    if (warp == kUProducer) {
+      produce_units<D, C>(smem, meta, full, empty, tmK, tmV, a, lane);
+      return;
+    }
 
-  if (warp == kUMma || warp == kUMma + 1) {
-    // ================================ MMA issuers (one per half) ==============================
-    const int h = warp - kUMma;
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, q_ph = 0, p_ph = 0, f_ph = 0;
-      const uint32_t q_base = pa::smem_addr(smem + C::kOffQ) + h * C::kQHalfBytes;
-      bool ok = true;
-      // One K = 16 step of S_h = Q_h K^T (k over d) and one K = 16 step of O_h += P_h V (i over the
-      // hi keys, then the lo keys).
-      auto s_step = [&](int st, int k) {
-        const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
-        const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
-        const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-        pa::umma_f16(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
-      };
-      auto pv_step = [&](int st, bool first_tile, int i) {
-        const int part = i / (kTile / 16), kk = i % (kTile / 16);
-        const uint32_t vb = pa::smem_addr(smem + st * C::kStageBytes) + C::kKVBytes;
-        const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
-        const bool init = first_tile && i == 0;
-        pa::umma_f16_tmem_a(tmem + 128 + D * h, tmem + kTmemP + 64 * h + part * 32 + kk * 8, db, kIdescO,
-                            init ? 0u : 1u);
-      };
-      constexpr int kPV = 2 * (kTile / 16);
-      while (ok) {
-        // first tile of a unit: S_h(0)
-        if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
-        Meta mt = meta[stage];
-        if (mt.flags & kDone) break;
-        if (!pa::mbar_wait(&q_ready[h], q_ph)) { ok = false; break; }
-        q_ph ^= 1;
-        pa::tc_fence_after();
-        // a half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
-        // MMAs, but its barriers are committed all the same so that both sides count the same phases
-        const bool active = h == 0 || mt.nq * G > kURows;
-        if (active) {
-#pragma unroll
-          for (int k = 0; k < KS; ++k) s_step(stage, k);
-        }
-        pa::umma_commit(&s_full[h]);
-        bool first = true;
-        while (true) {
-          const bool last = (mt.flags & kLast) != 0;
-          int nstage = stage + 1;
-          uint32_t nphase = phase;
-          if (nstage == C::kStages) {
-            nstage = 0;
-            nphase ^= 1;
+    if (warp >= kUMmaS && warp < kUMmaS + 2) {
+      // ================================ S issuers (one per half) ================================
+      const int h = warp - kUMmaS;
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0, q_ph = 0, f_ph = 0;
+        const uint32_t q_base = pa::smem_addr(smem + C::kOffQ) + h * C::kQHalfBytes;
+        bool ok = true;
+        // S_h = Q_h K^T over d in K = 16 steps
+        auto s_tile = [&](int st) {
+          const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
+  #pragma unroll
+          for (int k = 0; k < KS; ++k) {
+            const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
+            const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
+            pa::umma_f16_ss(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
           }
-          // S_h(j+1) as soon as the rows have read S_h(j) out of TMEM: it then runs during their
-          // softmax of tile j, and only P.V(j) waits for P
-          if (!pa::mbar_wait(&s_free[h], f_ph)) { ok = false; break; }
-          f_ph ^= 1;
-          if (!last) {
-            if (!pa::mbar_wait(&full[nstage], nphase)) { ok = false; break; }
-            pa::tc_fence_after();
-            if (active) {
-#pragma unroll
-              for (int k = 0; k < KS; ++k) s_step(nstage, k);
+        };
+        while (ok) {
+          // first tile of a unit: S_h(0) once the rows have staged the unit's Q
+          if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+          Meta mt = meta[stage];
+          if (mt.flags & kDone) break;
+          if (!pa::mbar_wait(&q_ready[h], q_ph)) { ok = false; break; }
+          q_ph ^= 1;
+          pa::tc_fence_after();
+          // a half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
+          // MMAs, but its barriers are committed all the same so that both sides count the same phases
+          const bool active = h == 0 || mt.nq * G > kURows;
+          if (active) s_tile(stage);
+          pa::umma_commit(&s_full[h]);
+          pa::umma_commit(&empty[stage]);  // this half is done with the stage's K once S_h has run
+          while (true) {
+            const bool last = (mt.flags & kLast) != 0;
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1;
             }
+            // S_h(j+1) as soon as the rows have read S_h(j) out of TMEM: it then runs during their
+            // softmax of tile j
+            if (!pa::mbar_wait(&s_free[h], f_ph)) { ok = false; break; }
+            f_ph ^= 1;
+            if (last) break;
+            if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+            pa::tc_fence_after();
+            mt = meta[stage];
+            if (active) s_tile(stage);
             pa::umma_commit(&s_full[h]);
+            pa::umma_commit(&empty[stage]);
           }
+        }
+        if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      }
+      if (h == 1) return;
+      __syncwarp();
+      // free TMEM once the row threads are done with it (they wait for every MMA's result)
+      pa::mbar_wait(teardown, 0);
+      pa::tc_fence_after();
+      pa::tmem_dealloc(tmem, kTmemCols);
+      return;
+    }
+
+    if (warp >= kUMmaPV && warp < kUMmaPV + 2) {
+      // ================================ P.V issuers (one per half) ==============================
+      const int h = warp - kUMmaPV;
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0, p_ph = 0;
+        bool ok = true;
+        constexpr int kPV = 2 * (kTile / 16);
+        while (ok) {
+          if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+          const Meta mt = meta[stage];
+          if (mt.flags & kDone) break;
+          const bool active = h == 0 || mt.nq * G > kURows;
+          const bool first = (mt.flags & kFirst) != 0;
+          // O_h += P_h V: i over the hi keys, then the lo keys, in K = 16 steps; A = P_h from TMEM
           if (!pa::mbar_wait(&p_full[h], p_ph)) { ok = false; break; }
           p_ph ^= 1;
           pa::tc_fence_after();
           if (active) {
-#pragma unroll
-            for (int i = 0; i < kPV; ++i) pv_step(stage, first, i);
+            const uint32_t vb = pa::smem_addr(smem + stage * C::kStageBytes) + C::kKVBytes;
+  #pragma unroll
+            for (int i = 0; i < kPV; ++i) {
+              const int part = i / (kTile / 16), kk = i % (kTile / 16);
+              const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
+              pa::umma_f16_tmem_a(tmem + 128 + D * h, tmem + kTmemP + 64 * h + part * 32 + kk * 8, db, kIdescO,
+                                  (first && i == 0) ? 0u : 1u);
+            }
           }
           pa::umma_commit(&o_done[h]);
-          pa::umma_commit(&empty[stage]);
-          stage = nstage;
-          phase = nphase;
-          if (last) break;
-          mt = meta[stage];
-          first = false;
+          pa::umma_commit(&empty[stage]);  // and with the stage's V once P_h V has run
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
+        if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
       }
-      if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      return;
     }
-    if (h == 1) return;
-    __syncwarp();
-    // free TMEM once the row threads are done with it
-    pa::mbar_wait(teardown, 0);
-    pa::tc_fence_after();
-    pa::tmem_dealloc(tmem, kTmemCols);
+
     return;
-  }
+  }  // warps 8-15
 
   // ================================== row threads (warps 0-7) =====================================
+  pa::setmaxnreg_inc<kRegsRows>();
   const int half = warp >> 2;                         // 0: rows 0..127, 1: rows 128..255
   const int hr = (warp & 3) * 32 + lane;              // row within the half = TMEM lane
   const int r = half * kURows + hr;                   // row within the unit
@@ -878,9 +908,16 @@ cudaError_t launch_umma(const CUtensorMap& tk, const CUtensorMap& tv, const Args
   using C = UCfg<D>;
   static bool ready = false;
   if (!ready) {
-    const cudaError_t e = cudaFuncSetAttribute(prefill_umma_kernel<T, D, G>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(prefill_umma_kernel<T, D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // The warpgroups' register split must fit in what the CTA is launched with, or the row
+    // warpgroups' setmaxnreg.inc would wait for ever: refuse to launch otherwise.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, prefill_umma_kernel<T, D, G>);
+    if (e != cudaSuccess) return e;
+    if (static_cast<long long>(fa.numRegs) * kUThreads < 2LL * 128 * (kRegsRows + kRegsOther))
+      return cudaErrorInvalidConfiguration;
     ready = true;
   }
   int dev = 0, sms = 148;

@@ -217,9 +217,11 @@ def test_shared_prefix_reads_same_blocks(oracle_mod, consumer):
 # ---- combine, cache write, copy blocks ---------------------------------------------------------
 
 @pytest.mark.parametrize("d", [64, 128])
-def test_combine_matches_oracle(oracle_mod, d):
+@pytest.mark.parametrize("long", [False, True])   # True: more than 64 partitions (several warps per row)
+def test_combine_matches_oracle(oracle_mod, d, long):
     P = 64
-    lens = torch.tensor([1, 64, 65, 300, 0, 1000], dtype=torch.int32)
+    lens = torch.tensor([1, 64, 65, 300, 0, 6000 if long else 1000] + ([4160, 2111, 64 * 70] if long else []),
+                        dtype=torch.int32)
     case = W.paged_case("comb", lens, 8, 2, d, 16, torch.float32, 92)
     n_parts = int(math.ceil(int(lens.max()) / P))
     po, pm, pl = oracle_mod.partials(case.q, case.k_cache, case.v_cache, case.block_tables, lens, P, n_parts)
