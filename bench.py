@@ -722,7 +722,7 @@ def run_prefill(args, rank, world, local_rank):
     q_start = torch.tensor([0] + list(torch.tensor(nq).cumsum(0)), dtype=torch.int32, device=dev)
     q = torch.randn((int(q_start[-1]), H, d), generator=torch.Generator(device=dev).manual_seed(5), device=dev).to(dt)
     max_c, max_q = max(ctx), max(nq)
-    ws = torch.empty(api._native.load().pa_prefill_workspace_size(len(ctx), H, Hk, max_q), dtype=torch.uint8,
+    ws = torch.empty(api.prefill_workspace_size(len(ctx), H, Hk, d, max_c, max_q), dtype=torch.uint8,
                      device=dev)
     out = torch.empty_like(q)
     flops = sum(4 * d * H * sum(c - n + i + 1 for i in range(n)) for c, n in zip(ctx, nq))

@@ -248,11 +248,14 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int
  *                 error word (pa_workspace_error) has bit 1 set if a bounded wait gave up and
  *                 bit 2 if a size was cut to its bound
  *
- * Kernel: tcgen05 tensor cores with the S and O accumulators and P in tensor memory (default);
- * the environment variable PA_PREFILL_CONSUMER=mma_sync selects the mma.sync kernel instead.
- * Both give the same results within the tolerance (P is carried as two 16-bit parts).
+ * Kernels: sequences with two or more query tokens run on tcgen05 tensor cores with the S and O
+ * accumulators and P in tensor memory (default; the environment variable
+ * PA_PREFILL_CONSUMER=mma_sync selects the mma.sync kernel instead; both give the same results
+ * within the tolerance, P being carried as two 16-bit parts).  Sequences with exactly one query
+ * token -- the decode rows of a mixed batch -- are computed by pa_decode's kernels in the same call
+ * (the decode definition is the n_s = 1 case), which stream their context at the HBM rate.
  */
-size_t pa_prefill_workspace_size(int S, int H, int Hk, int max_q_len);
+size_t pa_prefill_workspace_size(int S, int H, int Hk, int d, int max_context_len, int max_q_len);
 
 pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
                      const void* k_cache, const void* v_cache, const int32_t* block_tables,

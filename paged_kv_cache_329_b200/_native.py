@@ -41,7 +41,7 @@ SIGNATURES = {
     "pa_decode_step": (I, [P, I, P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, I, F, I, I, P, SZ, P]),
     "pa_decode_noalloc": (I, [P, I, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P]),
     "pa_decode_default_partition": (I, [I, I, I]),
-    "pa_prefill_workspace_size": (SZ, [I, I, I, I]),
+    "pa_prefill_workspace_size": (SZ, [I, I, I, I, I, I]),
     "pa_prefill": (I, [P, I, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, SZ, P]),
     "pa_workspace_error": (I, [P, IP, P]),
     "pa_selftest_wait_timeout": (I, [ctypes.c_uint, P, P]),

@@ -127,6 +127,10 @@ def pa_decode_step(q, k_cache, v_cache, block_tables, context_lens, key, value, 
     return out
 
 
+def prefill_workspace_size(S, H, Hk, d, max_context_len, max_q_len) -> int:
+    return _native.load().pa_prefill_workspace_size(S, H, Hk, d, int(max_context_len), int(max_q_len))
+
+
 def pa_prefill(q, q_start, k_cache, v_cache, block_tables, context_lens, *, max_context_len, max_q_len,
                scale=None, out=None, out_dtype=None, workspace=None, stream=None):
     """Causal paged attention for several query tokens per sequence (prefill chunks and decode tokens
@@ -140,7 +144,7 @@ def pa_prefill(q, q_start, k_cache, v_cache, block_tables, context_lens, *, max_
     if out is None:
         out = torch.empty((T, H, d), dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
-        n = _native.load().pa_prefill_workspace_size(S, H, Hk, int(max_q_len))
+        n = prefill_workspace_size(S, H, Hk, d, max_context_len, max_q_len)
         workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)

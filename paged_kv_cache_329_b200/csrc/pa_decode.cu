@@ -58,7 +58,7 @@ constexpr size_t kHdrBytes = 256;
 enum : int { kFirst = 1, kLast = 2, kDone = 4, kSingle = 8 };
 
 struct __align__(16) StageMeta {
-  int s, kh, part, ntok, flags, pad0, pad1, pad2;
+  int s, kh, part, ntok, flags, orow, pad1, pad2;  // orow: the sequence's row of query and out
 };
 
 struct DecodeArgs {
@@ -72,6 +72,8 @@ struct DecodeArgs {
   float scale_log2;  // scale * log2(e)
   const int2* items;
   int* hdr;
+  int* err;               // error word (the header's, or another call's when decode serves it)
+  const int32_t* q_rows;  // row of query / out for sequence s (null: row s)
   float* part_o;
   float* part_m;
   float* part_l;
@@ -134,17 +136,23 @@ struct PlanSmem {
 // sequence then writes its items, except that a warp writes the whole-partition items of a
 // sequence that has more than 32 of them.
 __device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restrict__ lens, int S, int Hk, int P,
-                                           int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
+                                           int max_c, int2* __restrict__ items, int* __restrict__ hdr,
+                                           const int32_t* __restrict__ q_start = nullptr, int* err = nullptr) {
+  // With q_start, only sequences with exactly one query token (q_start[s+1] - q_start[s] == 1) get
+  // units (the others are some other kernel's), and a cut length is or-ed into *err instead of
+  // resetting the header's error word.
   const int tid = threadIdx.x, nt = blockDim.x;
   const int nb = min(P / kTileTokens, kBuckets);
   for (int b = tid; b < kBuckets; b += nt) sm.count[b] = 0;
   __syncthreads();
   bool clamped = false;
   for (int s = tid; s < S; s += nt) {
+    const bool mine = !q_start || q_start[s + 1] - q_start[s] == 1;
     const int raw = lens[s];
-    clamped |= raw > max_c;
-    const int c = min(max(raw, 0), max_c);
+    clamped |= mine && raw > max_c;
+    const int c = mine ? min(max(raw, 0), max_c) : -1;  // -1: not listed
     if (s < kPlanCache) sm.c_cache[s] = c;
+    if (!mine) continue;
     const int f = max(1, (c + P - 1) / P) - 1;  // whole partitions before the last one
     if (f > 0) atomicAdd(&sm.count[nb - 1], f * Hk);
     atomicAdd(&sm.count[tile_bucket(c - f * P, P)], Hk);
@@ -183,7 +191,9 @@ __device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restri
   // A thread per sequence takes its places and writes its last-partition items; a sequence with
   // more than 32 whole-partition items leaves those to a warp (below).
   for (int s = tid; s < S; s += nt) {
-    const int c = s < kPlanCache ? sm.c_cache[s] : min(max(lens[s], 0), max_c);
+    const int c = s < kPlanCache ? sm.c_cache[s]
+                                 : ((!q_start || q_start[s + 1] - q_start[s] == 1) ? min(max(lens[s], 0), max_c) : -1);
+    if (c < 0) continue;
     const int f = max(1, (c + P - 1) / P) - 1;
     if (f > 0) {
       const int base = atomicAdd(&sm.cursor[nb - 1], f * Hk);
@@ -210,17 +220,24 @@ __device__ __forceinline__ void build_plan(PlanSmem& sm, const int32_t* __restri
     for (int i = lane; i < f * Hk; i += 32) items[base + i] = make_int2(s, ((i % Hk) << 16) | (i / Hk));
   }
   const int any_clamped = __syncthreads_or(clamped);
-  if (tid == 0) hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
+  if (tid == 0) {
+    if (err) {
+      if (any_clamped) atomicOr(err, pa::kErrBadLength);
+    } else {
+      hdr[kHdrError] = any_clamped ? pa::kErrBadLength : 0;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ lens, int S, int Hk, int P,
-                                                            int max_c, int2* __restrict__ items, int* __restrict__ hdr) {
+                                                            int max_c, int2* __restrict__ items, int* __restrict__ hdr,
+                                                            const int32_t* __restrict__ q_start, int* err) {
   // Let the decode grid start its set-up now; wait for earlier work on the stream (it may have
   // written the lengths) before reading anything.
   pa::grid_dependency_launch();
   pa::grid_dependency_wait();
   __shared__ PlanSmem sm;
-  build_plan(sm, lens, S, Hk, P, max_c, items, hdr);
+  build_plan(sm, lens, S, Hk, P, max_c, items, hdr, q_start, err);
 }
 
 // ---- step prologue: copy-on-write copies, slot writes and the plan in one launch ---------------
@@ -522,7 +539,7 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
     pa::mbar_arrive(epi);
     const bool done = pa::mbar_wait(epi, epi_phase);
     epi_phase ^= 1;
-    if (!done && lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    if (!done && lane == 0) atomicOr(a.err, pa::kErrWaitTimeout);
     return done;
   };
   // ldmatrix row/chunk assignment of this lane (tile index = lane / 8)
@@ -536,7 +553,7 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
 
   while (true) {
     if (!pa::mbar_wait(&full[stage], phase)) {
-      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      if (lane == 0) atomicOr(a.err, pa::kErrWaitTimeout);
       return;
     }
     const StageMeta mt = meta[stage];
@@ -702,7 +719,8 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
       if (!epi_sync()) return;
       if (warp < 2) put(merge + warp * G * D, true);
       if (!epi_sync()) return;
-      const size_t row = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;
+      const size_t row = static_cast<size_t>(mt.orow) * a.H + static_cast<size_t>(mt.kh) * G;   // out
+      const size_t prow = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;   // partials
 #pragma unroll
       for (int i = 0; i < NMINE; ++i) {
         const int f = tid + i * kConsumerWarps * 32;
@@ -722,7 +740,7 @@ __device__ __forceinline__ void consume_mma(uint8_t* stages, uint8_t* qslots, St
             else
               pa::store_floats<__nv_bfloat16, 4>(static_cast<__nv_bfloat16*>(a.out) + (row + h) * D + dd, v);
           } else {
-            const size_t pidx = (row + h) * a.max_parts + mt.part;
+            const size_t pidx = (prow + h) * a.max_parts + mt.part;
             pa::store_floats<float, 4>(a.part_o + pidx * D + dd, v);
             if (dd == 0) {
               a.part_m[pidx] = outM[i] == -INFINITY ? -INFINITY : outM[i] * kLn2;
@@ -802,6 +820,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       }
       const int2 it = a.items[k];
       const int s = it.x, kh = it.y >> 16, part = it.y & 0xffff;
+      const int orow = a.q_rows ? a.q_rows[s] : s;
       const int c = min(max(a.lens[s], 0), a.max_c);
       const int n_parts = max(1, (c + a.P - 1) / a.P);
       const int t0 = part * a.P;
@@ -819,7 +838,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         if (lane < nblk) {
           phys = __ldg(bt_row + j0 + lane);
           if (phys < 0 || phys >= a.n_blocks) {
-            atomicOr(a.hdr + kHdrError, pa::kErrBadBlock);
+            atomicOr(a.err, pa::kErrBadBlock);
             phys = -1;  // a fully out-of-range box: the TMA unit fills it with zeros
           }
         }
@@ -831,6 +850,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           m.part = part;
           m.ntok = ntok;
           m.flags = (tile == 0 ? kFirst : 0) | (tile == ntiles - 1 ? kLast : 0) | (n_parts == 1 ? kSingle : 0);
+          m.orow = orow;
           meta[stage] = m;
           pa::mbar_arrive_expect_tx(&full[stage], bytes);
         }
@@ -851,7 +871,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         }
         if (tile == 0 && lane == 0) {
           const uint8_t* qsrc = static_cast<const uint8_t*>(a.q) +
-                                (static_cast<size_t>(s) * a.H + static_cast<size_t>(kh) * G) * D * C::kES;
+                                (static_cast<size_t>(orow) * a.H + static_cast<size_t>(kh) * G) * D * C::kES;
           pa::bulk_load(qslots + stage * C::kQSlot, qsrc, C::kQBytes, &full[stage]);
         }
         ++issued;
@@ -862,7 +882,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
       }
     }
     if (!ok) {
-      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      if (lane == 0) atomicOr(a.err, pa::kErrWaitTimeout);
       // Let every copy this warp started land before the CTA can exit.
       int st = stage;
       uint32_t ph = phase;
@@ -903,12 +923,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     pa::mbar_arrive(epi);
     const bool done = pa::mbar_wait(epi, epi_phase);
     epi_phase ^= 1;
-    if (!done && lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+    if (!done && lane == 0) atomicOr(a.err, pa::kErrWaitTimeout);
     return done;
   };
   while (true) {
     if (!pa::mbar_wait(&full[stage], phase)) {
-      if (lane == 0) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
+      if (lane == 0) atomicOr(a.err, pa::kErrWaitTimeout);
       return;
     }
     const StageMeta mt = meta[stage];
@@ -1124,7 +1144,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
               acc[h][k * E + e + 2] += v.z;
               acc[h][k * E + e + 3] += v.w;
             }
-        const size_t row = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;
+        const size_t row = static_cast<size_t>(mt.orow) * a.H + static_cast<size_t>(mt.kh) * G;  // out
+        const size_t prow = static_cast<size_t>(mt.s) * a.H + static_cast<size_t>(mt.kh) * G;  // partials
         if (mt.flags & kSingle) {
           float inv[G];
 #pragma unroll
@@ -1142,7 +1163,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
           for (int h = 0; h < G; ++h) one[h] = 1.f;
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const size_t pidx = (row + h) * a.max_parts + mt.part;
+            const size_t pidx = (prow + h) * a.max_parts + mt.part;
             float acc_h[1][AC];
 #pragma unroll
             for (int e = 0; e < AC; ++e) acc_h[0][e] = acc[h][e];
@@ -1172,7 +1193,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 }
 
 // ---- log-sum-exp combine -----------------------------------------------------------------------
-// WPR warps per (sequence, query head); lane owns D/32 consecutive dims.  With WPR > 1 the warps of
+// WPR warps per (sequence, query head); lane owns D/32 consecutive dims.  q_rows is null, or the
+// q_start of a mixed batch whose one-token sequences are merged here (output row q_start[s]).  With WPR > 1 the warps of
 // a row take interleaved batches of 32 partitions (batch b to warp b % WPR) and their sums are
 // added in a fixed order through shared memory, so that rows with many partitions keep more loads
 // in flight.  Sequences with fewer than min_parts partitions are skipped (the decode kernel
@@ -1184,7 +1206,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(OutT* __restri
                                                                   const float* __restrict__ part_m,
                                                                   const float* __restrict__ part_l,
                                                                   const int32_t* __restrict__ lens, int S, int H,
-                                                                  int max_parts, int P, int min_parts) {
+                                                                  int max_parts, int P, int min_parts,
+                                                                  const int32_t* __restrict__ q_rows) {
   // Partitions past max_parts are never read: a length that needs more is cut to max_parts * P.
   pa::grid_dependency_wait();  // launched right behind the decode grid: its partials must be complete
   constexpr int PER = D / 32;
@@ -1206,6 +1229,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(OutT* __restri
     np = min((c + P - 1) / P, max_parts);
     // empty context: zeros (the decode kernel already wrote them when min_parts > 1)
     write = np == 0 ? min_parts <= 1 : np >= min_parts;
+    // q_rows is a mixed batch's q_start: only its one-token sequences are this launch's
+    if (q_rows && q_rows[s + 1] - q_rows[s] != 1) write = false;
   }
   if (write && np > 0) {
     const float* pm = part_m + gw * max_parts;
@@ -1261,7 +1286,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(OutT* __restri
     }
   }
   if (!write) return;
-  OutT* o = out + gw * D + lane * PER;
+  const long long orow = q_rows ? static_cast<long long>(q_rows[gw / H]) * H + gw % H : gw;
+  OutT* o = out + orow * D + lane * PER;
   const float inv = den > 0.f ? 1.f / den : 0.f;
   float res[PER];
 #pragma unroll
@@ -1339,28 +1365,30 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 template <int D, int WPR>
 cudaError_t launch_combine_w(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
-                             const int32_t* lens, int S, int H, int max_parts, int P, int min_parts, cudaStream_t st) {
+                             const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
+                             const int32_t* q_rows, cudaStream_t st) {
   constexpr int kRowsPerCta = kCombineThreads / 32 / WPR;
   const long long rows = static_cast<long long>(S) * H;
   const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta)), block(kCombineThreads);
   if (grid.x == 0) return cudaSuccess;
   if (out_dtype == PA_F32)
     return launch_pdl(combine_kernel<float, D, WPR>, grid, block, 0, st, static_cast<float*>(out), po, pm, pl, lens, S,
-                      H, max_parts, P, min_parts);
+                      H, max_parts, P, min_parts, q_rows);
   if (out_dtype == PA_F16)
     return launch_pdl(combine_kernel<__half, D, WPR>, grid, block, 0, st, static_cast<__half*>(out), po, pm, pl, lens,
-                      S, H, max_parts, P, min_parts);
+                      S, H, max_parts, P, min_parts, q_rows);
   return launch_pdl(combine_kernel<__nv_bfloat16, D, WPR>, grid, block, 0, st, static_cast<__nv_bfloat16*>(out), po,
-                    pm, pl, lens, S, H, max_parts, P, min_parts);
+                    pm, pl, lens, S, H, max_parts, P, min_parts, q_rows);
 }
 
 // Rows with many partitions (more than two batches of 32) get four warps each.
 template <int D>
 cudaError_t launch_combine(void* out, pa_dtype out_dtype, const float* po, const float* pm, const float* pl,
                            const int32_t* lens, int S, int H, int max_parts, int P, int min_parts,
-                           cudaStream_t st) {
-  return max_parts > 64 ? launch_combine_w<D, 4>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, st)
-                        : launch_combine_w<D, 1>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, st);
+                           cudaStream_t st, const int32_t* q_rows = nullptr) {
+  return max_parts > 64
+             ? launch_combine_w<D, 4>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, q_rows, st)
+             : launch_combine_w<D, 1>(out, out_dtype, po, pm, pl, lens, S, H, max_parts, P, min_parts, q_rows, st);
 }
 
 struct DeviceInfo {
@@ -1549,6 +1577,8 @@ pa_status prepare_decode(DecodePlan& dp, const char* who, void* out, pa_dtype ou
   a.scale_log2 = scale * kLog2e;
   a.items = reinterpret_cast<const int2*>(ws + dp.wl.items);
   a.hdr = reinterpret_cast<int*>(ws);
+  a.err = a.hdr + kHdrError;
+  a.q_rows = nullptr;
   a.part_o = reinterpret_cast<float*>(ws + dp.wl.part_o);
   a.part_m = reinterpret_cast<float*>(ws + dp.wl.part_m);
   a.part_l = reinterpret_cast<float*>(ws + dp.wl.part_l);
@@ -1568,9 +1598,9 @@ pa_status launch_decode_and_combine(const DecodePlan& dp, const char* who, cudaS
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: decode launch failed: %s", who, cudaGetErrorString(e));
   if (dp.max_parts > 1) {
     e = dp.d == 64 ? launch_combine<64>(a.out, dp.out_dtype, a.part_o, a.part_m, a.part_l, a.lens, a.S, a.H,
-                                        dp.max_parts, dp.P, 2, st)
+                                        dp.max_parts, dp.P, 2, st, a.q_rows)
                    : launch_combine<128>(a.out, dp.out_dtype, a.part_o, a.part_m, a.part_l, a.lens, a.S, a.H,
-                                         dp.max_parts, dp.P, 2, st);
+                                         dp.max_parts, dp.P, 2, st, a.q_rows);
     if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "%s: combine launch failed: %s", who, cudaGetErrorString(e));
   }
   return pa::ok();
@@ -1591,9 +1621,50 @@ extern "C" pa_status pa_decode(void* out, pa_dtype out_dtype, const void* query,
   if (S == 0) return pa::ok();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, context_lens, S, Hk, dp.P,
-                                   max_context_len, reinterpret_cast<int2*>(const_cast<int2*>(dp.a.items)), dp.a.hdr);
+                                   max_context_len, reinterpret_cast<int2*>(const_cast<int2*>(dp.a.items)), dp.a.hdr,
+                                   static_cast<const int32_t*>(nullptr), static_cast<int*>(nullptr));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_decode: plan launch failed: %s", cudaGetErrorString(e));
   return launch_decode_and_combine(dp, "pa_decode", st);
+}
+
+// ---- decode of the one-token sequences of a mixed batch (for pa_prefill) ---------------------------
+// The sequences with exactly one query token are decoded by the kernels above: their query and
+// output rows are q_start[s], their units come from a plan that skips every other sequence, and
+// errors are or-ed into the caller's error word.
+
+namespace {
+int single_rows_partition(int S, int Hk, int max_context_len) {
+  const int P = default_partition(S, Hk, max_context_len);
+  return P > 1024 ? 1024 : P;
+}
+}  // namespace
+
+size_t pa::decode_single_rows_workspace(int S, int H, int Hk, int d, int max_context_len) {
+  return pa_decode_workspace_size(S, H, Hk, d, max_context_len, single_rows_partition(S, Hk, max_context_len));
+}
+
+pa_status pa::decode_single_rows(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
+                                 const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int S, int H, int Hk, int d, int B, int n_blocks,
+                                 int max_blocks_per_seq, int max_context_len, float scale, pa_dtype kv_dtype,
+                                 void* workspace, size_t workspace_bytes, int* err, void* stream) {
+  // A mixed batch's decode rows are usually a minority of its sequences, so the unit count that
+  // the default partition assumes (every sequence at max_context_len) overstates their work and
+  // the longest of them would be the grid's tail: partitions of at most 1024 tokens.
+  DecodePlan dp;
+  const pa_status ps = prepare_decode(dp, "pa_prefill (one-token rows)", out, out_dtype, query, k_cache, v_cache,
+                                      block_tables, context_lens, S, H, Hk, d, B, n_blocks, max_blocks_per_seq,
+                                      max_context_len, scale, kv_dtype, single_rows_partition(S, Hk, max_context_len),
+                                      workspace, workspace_bytes);
+  if (ps != PA_OK || S == 0) return ps;
+  dp.a.q_rows = q_start;
+  dp.a.err = err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, context_lens, S, Hk, dp.P,
+                                   max_context_len, reinterpret_cast<int2*>(const_cast<int2*>(dp.a.items)), dp.a.hdr,
+                                   q_start, err);
+  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: plan launch failed: %s", cudaGetErrorString(e));
+  return launch_decode_and_combine(dp, "pa_prefill (one-token rows)", st);
 }
 
 extern "C" pa_status pa_decode_step(void* out, pa_dtype out_dtype, const void* query, void* k_cache, void* v_cache,

@@ -343,6 +343,57 @@ struct Split<__half> {
   }
 };
 
+// ---- packed fp32 pairs (sm_100: one instruction operates on two floats) ----------------------------
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {  // a * b + c, rounded
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three floats in one instruction
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Split<T>::run for a pair already packed as p2 = {x0, x1}: the bf16 form subtracts the cut-off hi
+// parts from both in one packed instruction.
+template <class T>
+struct Split2 {
+  __device__ __forceinline__ static void run(float x0, float x1, uint64_t, uint32_t& hi, uint32_t& lo) {
+    Split<T>::run(x0, x1, hi, lo);
+  }
+};
+template <>
+struct Split2<__nv_bfloat16> {
+  __device__ __forceinline__ static void run(float x0, float x1, uint64_t p2, uint32_t& hi, uint32_t& lo) {
+    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(hi) : "r"(b0), "r"(b1));
+    const uint64_t l2 = f2_sub(p2, f2_pack(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u)));
+    float l0, l1;
+    f2_unpack(l2, l0, l1);
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(lo) : "r"(__float_as_uint(l0)), "r"(__float_as_uint(l1)));
+  }
+};
+
 // Store 32 consecutive 32-bit columns of this warp's 32 lanes; complete (visible to the tensor
 // core after a thread sync) once tmem_wait_st returns.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {

@@ -25,4 +25,15 @@ constexpr int kMaxStepPairs = 8192;
 pa_status copy_blocks_counted(void* k_cache, void* v_cache, const int32_t* pairs, const int32_t* n_pairs_dev,
                               int max_pairs, int Hk, int d, int B, int n_blocks, pa_dtype dtype, void* stream);
 
+// Decode attention of the sequences of a mixed batch that have exactly one query token
+// (q_start[s+1] - q_start[s] == 1): query and output row q_start[s], the decode kernels of
+// pa_decode, a cut length or a kernel error or-ed into *err (a device int).  The workspace is
+// decode_single_rows_workspace(...) bytes, 256-byte aligned.
+size_t decode_single_rows_workspace(int S, int H, int Hk, int d, int max_context_len);
+pa_status decode_single_rows(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
+                             const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, int S, int H, int Hk, int d, int B, int n_blocks,
+                             int max_blocks_per_seq, int max_context_len, float scale, pa_dtype kv_dtype,
+                             void* workspace, size_t workspace_bytes, int* err, void* stream);
+
 }  // namespace pa

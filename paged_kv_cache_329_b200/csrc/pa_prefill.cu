@@ -58,6 +58,7 @@ struct Args {
   const int32_t* bt;
   const int32_t* lens;
   int S, H, Hk, max_blocks, n_blocks, B, max_c, max_q, QT;
+  int route_single;  // sequences with one query token are left to the decode kernels
   float scale_log2;
   const int2* items;
   int* hdr;
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(Args a, int2
     bool bad;
     seq_sizes(a, s, n, c, bad);
     bad_any |= bad;
+    if (a.route_single && n == 1) continue;
     for (int t0 = 0; t0 < n; t0 += a.QT) atomicAdd(&count[bucket_of(c - n + min(t0 + a.QT, n), a.max_c)], a.Hk);
   }
   __syncthreads();
@@ -121,6 +123,7 @@ __global__ void __launch_bounds__(kPlanThreads) prefill_plan_kernel(Args a, int2
     int n, c;
     bool bad;
     seq_sizes(a, s, n, c, bad);
+    if (a.route_single && n == 1) continue;
     for (int t0 = 0, qt = 0; t0 < n; t0 += a.QT, ++qt) {
       const int base = atomicAdd(&cursor[bucket_of(c - n + min(t0 + a.QT, n), a.max_c)], a.Hk);
       for (int kh = 0; kh < a.Hk; ++kh) items[base + kh] = make_int2(s, (kh << 16) | qt);
@@ -754,13 +757,16 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < kTile; ++c) sv[c] = c < cut ? sv[c] : -INFINITY;
       }
-      float mx8[8];
+      // row maximum with three-input max: 64 -> 22 -> 8 -> 3 -> 1
+      float m22[22];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+      for (int i = 0; i < 21; ++i) m22[i] = pa::max3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
+      m22[21] = sv[63];
+      float m8[8];
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+      for (int i = 0; i < 7; ++i) m8[i] = pa::max3(m22[3 * i], m22[3 * i + 1], m22[3 * i + 2]);
+      m8[7] = m22[21];
+      const float mx = pa::max3(pa::max3(m8[0], m8[1], m8[2]), pa::max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
       // the running maximum moves only when it grows by more than 2^8; O is then rescaled by f
       // (below, once P.V(j-1) is done), decided per warp because tcgen05.ld/st are warp-collective
       if (mx > m_used + 8.f) {
@@ -771,15 +777,22 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       rescale = !(mt.flags & kFirst) && __any_sync(0xffffffffu, f != 1.f);
       // p = 2^(s * sl2 - m); with no visible key so far every s is -inf and p = 0
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // two keys per packed instruction for the scaling, the row sum and the lo parts
+      const uint64_t sc2 = pa::f2_pack(sl2, sl2), nm2 = pa::f2_pack(neg_m, neg_m);
+      uint64_t ls2[2] = {pa::f2_pack(0.f, 0.f), pa::f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int k2 = 0; k2 < kTile / 2; ++k2) {
-        const float p0 = pa::ex2(fmaf(sv[2 * k2], sl2, neg_m));
-        const float p1 = pa::ex2(fmaf(sv[2 * k2 + 1], sl2, neg_m));
-        ls[k2 & 3] += p0 + p1;
-        pa::Split<T>::run(p0, p1, hi[k2], lo[k2]);
+        float x0, x1;
+        pa::f2_unpack(pa::f2_fma(pa::f2_pack(sv[2 * k2], sv[2 * k2 + 1]), sc2, nm2), x0, x1);
+        const float p0 = pa::ex2(x0), p1 = pa::ex2(x1);
+        const uint64_t p2 = pa::f2_pack(p0, p1);
+        ls2[k2 & 1] = pa::f2_add(ls2[k2 & 1], p2);
+        pa::Split2<T>::run(p0, p1, p2, hi[k2], lo[k2]);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float l0, l1, l2v, l3;
+      pa::f2_unpack(ls2[0], l0, l1);
+      pa::f2_unpack(ls2[1], l2v, l3);
+      l += (l0 + l1) + (l2v + l3);
     }
     // P.V(j-1) must be complete before P is rewritten and O rescaled
     if (pv_pending) {
@@ -956,11 +969,16 @@ cudaError_t dispatch(int g, const CUtensorMap& tk, const CUtensorMap& tv, const 
   }
 }
 
+// The prefill kernel's header and unit list, then the decode workspace of the one-token sequences.
+size_t prefill_part_bytes(int S, int H, int Hk, int max_q_len) {
+  return align_up(kHdrBytes + sizeof(int2) * max_units(S, Hk, H / Hk, max_q_len), 256);
+}
+
 }  // namespace
 
-extern "C" size_t pa_prefill_workspace_size(int S, int H, int Hk, int max_q_len) {
-  if (S < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || max_q_len < 0) return 0;
-  return align_up(kHdrBytes + sizeof(int2) * max_units(S, Hk, H / Hk, max_q_len), 256);
+extern "C" size_t pa_prefill_workspace_size(int S, int H, int Hk, int d, int max_context_len, int max_q_len) {
+  if (S < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || max_q_len < 0 || max_context_len < 0 || d <= 0) return 0;
+  return prefill_part_bytes(S, H, Hk, max_q_len) + pa::decode_single_rows_workspace(S, H, Hk, d, max_context_len);
 }
 
 extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query, const int32_t* q_start,
@@ -990,7 +1008,7 @@ extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query
   if (!pa::aligned16(out) || !pa::aligned16(query) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
     return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: tensors must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: workspace must be 256-byte aligned");
-  const size_t need = pa_prefill_workspace_size(S, H, Hk, max_q_len);
+  const size_t need = pa_prefill_workspace_size(S, H, Hk, d, max_context_len, max_q_len);
   if (workspace_bytes < need) return pa::fail(PA_ERR_INVALID_ARG, "pa_prefill: workspace of %zu bytes < %zu needed", workspace_bytes, need);
   CUtensorMap tk, tv;
   if (!cache_map(&tk, k_cache, kv_dtype, d, rows, B) || !cache_map(&tv, v_cache, kv_dtype, d, rows, B))
@@ -1012,6 +1030,7 @@ extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query
   a.max_q = max_q_len;
   a.QT = rows_per_unit() / g;  // the workspace is sized for the smaller unit (more units)
   a.scale_log2 = scale * kLog2e;
+  a.route_single = 1;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.hdr = reinterpret_cast<int*>(ws);
   a.items = reinterpret_cast<const int2*>(ws + kHdrBytes);
@@ -1019,11 +1038,18 @@ extern "C" pa_status pa_prefill(void* out, pa_dtype out_dtype, const void* query
   cudaError_t e = launch_pdl(prefill_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, a,
                              reinterpret_cast<int2*>(ws + kHdrBytes));
   if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: plan launch failed: %s", cudaGetErrorString(e));
-  if (kv_dtype == PA_F16)
-    e = d == 64 ? dispatch<__half, 64>(g, tk, tv, a, units, st) : dispatch<__half, 128>(g, tk, tv, a, units, st);
-  else
-    e = d == 64 ? dispatch<__nv_bfloat16, 64>(g, tk, tv, a, units, st)
-                : dispatch<__nv_bfloat16, 128>(g, tk, tv, a, units, st);
-  if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s", cudaGetErrorString(e));
-  return pa::ok();
+  if (max_q_len > 1) {  // with at most one query token per sequence the decode kernels do all of it
+    if (kv_dtype == PA_F16)
+      e = d == 64 ? dispatch<__half, 64>(g, tk, tv, a, units, st) : dispatch<__half, 128>(g, tk, tv, a, units, st);
+    else
+      e = d == 64 ? dispatch<__nv_bfloat16, 64>(g, tk, tv, a, units, st)
+                  : dispatch<__nv_bfloat16, 128>(g, tk, tv, a, units, st);
+    if (e != cudaSuccess) return pa::fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s", cudaGetErrorString(e));
+  }
+  // The sequences with one query token (decode rows of a mixed batch): the decode kernels, which
+  // stream their context at the HBM rate instead of spending a 128-row tensor-core tile on g rows.
+  const size_t off = prefill_part_bytes(S, H, Hk, max_q_len);
+  return pa::decode_single_rows(out, out_dtype, query, q_start, k_cache, v_cache, block_tables, context_lens, S, H, Hk,
+                                d, B, n_blocks, max_blocks_per_seq, max_context_len, scale, kv_dtype, ws + off,
+                                workspace_bytes - off, a.hdr + kHdrError, stream);
 }

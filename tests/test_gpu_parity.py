@@ -498,7 +498,7 @@ def test_prefill_mixed_batch(oracle_mod, dtype, g, d, B):
     ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
                              case.scale, n_threads=0)
     dev = case.to("cuda")
-    ws = torch.empty(api._native.load().pa_prefill_workspace_size(case.S, case.H, Hk, max(nq)), dtype=torch.uint8,
+    ws = torch.empty(api.prefill_workspace_size(case.S, case.H, Hk, d, max(ctx), max(nq)), dtype=torch.uint8,
                      device="cuda")
     out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables, dev.context_lens,
                          max_context_len=max(ctx), max_q_len=max(nq), scale=case.scale, out_dtype=torch.float32,
