@@ -237,19 +237,29 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
+def code_sha256(path):
+    """sha256 of a C/C++/CUDA source with its comments and blank lines removed, so that a comment
+    edit does not count as a change of the code a profile was taken on."""
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.split("\n")]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
+
+
 def profiled_traffic(args):
-    """DRAM bytes per decode launch from the committed ncu summary, if its source hash matches and
-    the run is the workload it was captured on (gqa8k_bf16, library-default partition and B)."""
+    """DRAM bytes per decode launch from the committed ncu summary, if the code it was captured on
+    is the current code (comments aside) and the run is the workload it was captured on
+    (gqa8k_bf16, library-default partition and B, all sequences)."""
     if args.workload != "gqa8k_bf16" or args.partition or args.block_size or args.seqs:
         return None
     path = os.path.join(ROOT, "profiles", "decode_kernel_gqa8k_bf16.md")
-    src = os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", "pa_decode.cu")
+    srcs = [os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", f) for f in ("pa_decode.cu", "pa_device.cuh")]
     try:
         text = open(path).read()
-        h = re.search(r"source_sha256:\s*([0-9a-f]{64})", text).group(1)
+        want = dict(re.findall(r"code_sha256\((\S+)\):\s*([0-9a-f]{64})", text))
         t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text).group(1)
-        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        return float(t) if h == cur else None
+        ok = all(want.get(os.path.basename(f)) == code_sha256(f) for f in srcs)
+        return float(t) if ok else None
     except Exception:
         return None
 

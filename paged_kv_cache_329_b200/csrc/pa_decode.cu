@@ -11,9 +11,9 @@
 //   * Work unit = (sequence, kv head, partition of P tokens).  A plan kernel lists the units
 //     (whole partitions first, then the tails); a persistent grid pulls them from an atomic
 //     counter, so long and short sequences balance across the 148 SMs.
-//   * Per CTA one producer warp streams 64-token tiles of K and V into shared memory with 2-D TMA
-//     loads (one box per physical block and 128-byte column panel, 128-byte swizzle), into a ring
-//     of stages guarded by full/empty mbarriers.  The q rows of the unit's head group come in with
+//   * Per CTA one producer warp streams 64-token tiles of K and V into shared memory with TMA
+//     loads (one box per physical block holding all its 128-byte column panels, 128-byte
+//     swizzle), into a ring of stages guarded by full/empty mbarriers.  The q rows of the unit's head group come in with
 //     the first tile by a 1-D bulk copy.  Each block is located through the block table, so the
 //     kernel never touches a slot past the sequence's length.
 //   * Four consumer warps share every loaded tile across the g = H/Hk query heads of the group.
@@ -25,6 +25,9 @@
 //     memory in a fixed order, then write the final row (single-partition sequences) or the
 //     partial state for the combine kernel.  All summation orders depend only on logical token
 //     positions, so outputs do not change when blocks move to other physical ids.
+//   * pa_decode_step puts a step's copy-on-write copies, slot writes and the plan into one
+//     prologue kernel ahead of the decode grid ("PagedAttention原理", "解决COW": copy, then write,
+//     then read), and pa_prefill hands its one-token sequences to these kernels (rows q_start[s]).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
