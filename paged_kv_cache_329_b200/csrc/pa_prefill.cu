@@ -471,14 +471,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 // cycles with A in shared memory and 166-186 with A in tensor memory, whatever its N up to 128
 // (measured on B200), and separate issuing warps add up: four issuers keep up with the tensor core
 // where one per half (about 2400 issue cycles per 64-key tile) did not.  Warp 9 also allocates TMEM.
-// Per 64-key tile j and half h:
-//   S_h[128 x 64]  = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
-//   the rows of h read S_h from TMEM, mask causally, write P_h (hi and lo 16-bit parts) back to TMEM
-//   O_h[128 x d]  += P_h,hi V_j + P_h,lo V_j    A = P_h from TMEM, B = V tile (MN-major: d contiguous)
-// The halves are independent pipelines that share the K/V ring.  S_h(j+1) is issued as soon as the
-// rows have read S_h(j) out of TMEM, so it runs during their softmax of tile j and only P.V(j) waits
-// for P.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only
-// when a row's maximum grows by more than 2^8, which keeps every exponent bounded.
+// Per 64-key tile j and half h, in the TMEM buffer b = j mod 2 of that half:
+//   S_h,b[128 x 64] = Q_h K_j^T              d/16 tcgen05.mma, A = Q tile, B = K tile (K-major)
+//   the rows of h read S out of the buffer, mask causally, and write P (hi and lo 16-bit parts) back
+//   into the same 64 columns
+//   O_h[128 x d]  += P_hi V_j + P_lo V_j      A = P from TMEM, B = V tile (MN-major: d contiguous)
+// The halves are independent pipelines that share the K/V ring.  With two buffers per half the
+// rows never wait for a P.V product before writing P (P(j) replaces S(j), which they have just
+// read); S(j+2) waits until P.V(j) has read P(j) out of buffer b, so S(j+1) is ready while the rows
+// still work on tile j.  The running maximum is updated lazily: O_h (in TMEM) is rescaled only when
+// a row's maximum grows by more than 2^8, which keeps every exponent bounded; only then do the rows
+// wait for P.V(j-1).
 constexpr int kURows = 128;                  // rows per half (TMEM lanes)
 constexpr int kUHalves = 2;
 constexpr int kUUnitRows = kURows * kUHalves;
@@ -491,8 +494,8 @@ constexpr int kUThreads = 16 * 32;          // four warpgroups: rows (2), produc
 // 512 x 128, or the raise would wait for registers that are never released.
 constexpr uint32_t kRegsRows = 200, kRegsOther = 56;
 static_assert(2 * 128 * (kRegsRows + kRegsOther) <= 512 * 128, "register split exceeds the launch allocation");
-constexpr uint32_t kTmemCols = 512;          // S_A 0..63, S_B 64..127, O_A 128.., O_B 128+d.., P_A 384.., P_B 448..
-constexpr uint32_t kTmemP = 384;             // P_h: 32 columns of packed hi pairs, then 32 of lo pairs
+constexpr uint32_t kTmemCols = 512;          // S/P buffers 64 (2h + b).., O_A 256.., O_B 256 + d..
+constexpr uint32_t kTmemO = 256;             // P in a buffer: 32 columns of packed hi pairs, then 32 of lo pairs
 
 template <int D>
 struct UCfg {
@@ -506,12 +509,12 @@ struct UCfg {
   static constexpr int kOffQ = kStages * kStageBytes;
   static constexpr int kOffMeta = kOffQ + kUHalves * kQHalfBytes;
   static constexpr int kOffBar = kOffMeta + kStages * static_cast<int>(sizeof(Meta));
-  // full[S], empty[S], then per half: q_ready, s_full, p_full, o_done, s_free; then teardown
-  static constexpr int kNBars = 2 * kStages + 5 * kUHalves + 1;
+  // full[S], empty[S], q_ready[2], then per (half, buffer): s_full, p_full, o_done; then teardown
+  static constexpr int kNBars = 2 * kStages + kUHalves + 3 * 2 * kUHalves + 1;
   static constexpr int kOffTmem = kOffBar + kNBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(128 + kUHalves * D <= static_cast<int>(kTmemP), "TMEM columns: two S tiles and two O tiles below P");
+  static_assert(kTmemO + kUHalves * D <= static_cast<int>(kTmemCols), "TMEM columns: four S/P buffers and two O tiles");
 };
 
 template <class T, int D, int G>
@@ -528,12 +531,13 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + C::kStages;
+  // per (half h, buffer b) at index 2h + b: barriers of one buffer complete once every two tiles,
+  // so no waiter can fall two phases behind (tile j + 2 of a buffer needs tile j's P.V first)
   uint64_t* q_ready = empty + C::kStages;      // [2]
-  uint64_t* s_full = q_ready + kUHalves;       // [2]
-  uint64_t* p_full = s_full + kUHalves;        // [2]
-  uint64_t* o_done = p_full + kUHalves;        // [2]
-  uint64_t* s_free = o_done + kUHalves;        // [2]: the rows of h have read S_h out of TMEM
-  uint64_t* teardown = s_free + kUHalves;
+  uint64_t* s_full = q_ready + kUHalves;       // [4]: S(j) is in the buffer
+  uint64_t* p_full = s_full + 2 * kUHalves;    // [4]: the rows have written P(j) into it
+  uint64_t* o_done = p_full + 2 * kUHalves;    // [4]: P.V(j) has run (the buffer is free, O is current)
+  uint64_t* teardown = o_done + 2 * kUHalves;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -541,12 +545,11 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       pa::mbar_init(&full[i], 1);
       pa::mbar_init(&empty[i], 2 * kUHalves);  // one tcgen05.commit per tile from each of the 4 issuers
     }
-    for (int h = 0; h < kUHalves; ++h) {
-      pa::mbar_init(&q_ready[h], kURows);
-      pa::mbar_init(&s_full[h], 1);
-      pa::mbar_init(&p_full[h], kURows);
-      pa::mbar_init(&o_done[h], 1);
-      pa::mbar_init(&s_free[h], kURows);
+    for (int h = 0; h < kUHalves; ++h) pa::mbar_init(&q_ready[h], kURows);
+    for (int i = 0; i < 2 * kUHalves; ++i) {
+      pa::mbar_init(&s_full[i], 1);
+      pa::mbar_init(&p_full[i], kURows);
+      pa::mbar_init(&o_done[i], 1);
     }
     pa::mbar_init(teardown, kUUnitRows);
     pa::fence_barrier_init();
@@ -576,50 +579,42 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       const int h = warp - kUMmaS;
       if (lane == 0) {
         int stage = 0;
-        uint32_t phase = 0, q_ph = 0, f_ph = 0;
+        uint32_t phase = 0, q_ph = 0;
         const uint32_t q_base = pa::smem_addr(smem + C::kOffQ) + h * C::kQHalfBytes;
-        bool ok = true;
-        // S_h = Q_h K^T over d in K = 16 steps
-        auto s_tile = [&](int st) {
+        bool ok = true, active = false;
+        // S = Q_h K^T over d in K = 16 steps, into buffer b of this half
+        auto s_tile = [&](int st, int b) {
           const uint32_t kb = pa::smem_addr(smem + st * C::kStageBytes);
   #pragma unroll
           for (int k = 0; k < KS; ++k) {
             const uint64_t da = pa::sw128_desc(q_base + (k >> 2) * C::kQPanelBytes + (k & 3) * 32, 16, 1024);
             const uint64_t db = pa::sw128_desc(kb + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-            pa::umma_f16_ss(tmem + 64 * h, da, db, kIdescS, k > 0 ? 1u : 0u);
+            pa::umma_f16_ss(tmem + 64 * (2 * h + b), da, db, kIdescS, k > 0 ? 1u : 0u);
           }
         };
-        while (ok) {
-          // first tile of a unit: S_h(0) once the rows have staged the unit's Q
+        // n counts this half's tiles over all units of the CTA; tile n uses buffer n & 1
+        for (uint32_t n = 0;; ++n) {
           if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
-          Meta mt = meta[stage];
+          const Meta mt = meta[stage];
           if (mt.flags & kDone) break;
-          if (!pa::mbar_wait(&q_ready[h], q_ph)) { ok = false; break; }
-          q_ph ^= 1;
+          if (mt.flags & kFirst) {
+            // the unit's Q, staged by the rows once they have read the previous unit's last S
+            if (!pa::mbar_wait(&q_ready[h], q_ph)) { ok = false; break; }
+            q_ph ^= 1;
+            // a half whose rows hold no query (a short unit, a ragged chunk end) gets no MMAs, but
+            // its barriers are committed all the same so that both sides count the same phases
+            active = h == 0 || mt.nq * G > kURows;
+          }
+          const int b = static_cast<int>(n & 1u);
+          // the buffer is free once P.V(n - 2) has read its P
+          if (n >= 2 && !pa::mbar_wait(&o_done[2 * h + b], ((n - 2) >> 1) & 1u)) { ok = false; break; }
           pa::tc_fence_after();
-          // a half whose rows hold no query (a short unit: decode tokens, a ragged chunk end) gets no
-          // MMAs, but its barriers are committed all the same so that both sides count the same phases
-          const bool active = h == 0 || mt.nq * G > kURows;
-          if (active) s_tile(stage);
-          pa::umma_commit(&s_full[h]);
-          pa::umma_commit(&empty[stage]);  // this half is done with the stage's K once S_h has run
-          while (true) {
-            const bool last = (mt.flags & kLast) != 0;
-            if (++stage == C::kStages) {
-              stage = 0;
-              phase ^= 1;
-            }
-            // S_h(j+1) as soon as the rows have read S_h(j) out of TMEM: it then runs during their
-            // softmax of tile j
-            if (!pa::mbar_wait(&s_free[h], f_ph)) { ok = false; break; }
-            f_ph ^= 1;
-            if (last) break;
-            if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
-            pa::tc_fence_after();
-            mt = meta[stage];
-            if (active) s_tile(stage);
-            pa::umma_commit(&s_full[h]);
-            pa::umma_commit(&empty[stage]);
+          if (active) s_tile(stage, b);
+          pa::umma_commit(&s_full[2 * h + b]);
+          pa::umma_commit(&empty[stage]);  // this half is done with the stage's K once S has run
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
           }
         }
         if (!ok) atomicOr(a.hdr + kHdrError, pa::kErrWaitTimeout);
@@ -638,18 +633,18 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       const int h = warp - kUMmaPV;
       if (lane == 0) {
         int stage = 0;
-        uint32_t phase = 0, p_ph = 0;
+        uint32_t phase = 0;
         bool ok = true;
         constexpr int kPV = 2 * (kTile / 16);
-        while (ok) {
+        for (uint32_t n = 0;; ++n) {
           if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
           const Meta mt = meta[stage];
           if (mt.flags & kDone) break;
           const bool active = h == 0 || mt.nq * G > kURows;
           const bool first = (mt.flags & kFirst) != 0;
-          // O_h += P_h V: i over the hi keys, then the lo keys, in K = 16 steps; A = P_h from TMEM
-          if (!pa::mbar_wait(&p_full[h], p_ph)) { ok = false; break; }
-          p_ph ^= 1;
+          const int b = static_cast<int>(n & 1u);
+          // O_h += P V: i over the hi keys, then the lo keys, in K = 16 steps; A = P from buffer b
+          if (!pa::mbar_wait(&p_full[2 * h + b], (n >> 1) & 1u)) { ok = false; break; }
           pa::tc_fence_after();
           if (active) {
             const uint32_t vb = pa::smem_addr(smem + stage * C::kStageBytes) + C::kKVBytes;
@@ -657,12 +652,12 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
             for (int i = 0; i < kPV; ++i) {
               const int part = i / (kTile / 16), kk = i % (kTile / 16);
               const uint64_t db = pa::sw128_desc(vb + kk * 16 * 128, C::kPanelBytes, 1024);
-              pa::umma_f16_tmem_a(tmem + 128 + D * h, tmem + kTmemP + 64 * h + part * 32 + kk * 8, db, kIdescO,
+              pa::umma_f16_tmem_a(tmem + kTmemO + D * h, tmem + 64 * (2 * h + b) + part * 32 + kk * 8, db, kIdescO,
                                   (first && i == 0) ? 0u : 1u);
             }
           }
-          pa::umma_commit(&o_done[h]);
-          pa::umma_commit(&empty[stage]);  // and with the stage's V once P_h V has run
+          pa::umma_commit(&o_done[2 * h + b]);
+          pa::umma_commit(&empty[stage]);  // and with the stage's V once P V has run
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
@@ -683,19 +678,20 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   const int r = half * kURows + hr;                   // row within the unit
   const int warp_row0 = half * kURows + (warp & 3) * 32;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tS = tmem + 64 * half, tO = tmem + 128 + D * half, tP = tmem + kTmemP + 64 * half;
+  const uint32_t tSP = tmem + 64 * (2 * half), tO = tmem + kTmemO + D * half;
   uint8_t* qs = smem + C::kOffQ + half * C::kQHalfBytes;
   uint64_t* my_q_ready = &q_ready[half];
-  uint64_t* my_s_full = &s_full[half];
-  uint64_t* my_p_full = &p_full[half];
-  uint64_t* my_o_done = &o_done[half];
   int stage = 0;
-  uint32_t phase = 0, s_ph = 0, o_ph = 0;
+  uint32_t phase = 0;
   float m_used = -INFINITY, l = 0.f;
   int row_global = -1, qpos = 0;
-  bool pv_pending = false, ok = true, warp_active = false;
+  bool ok = true, warp_active = false;
   const float sl2 = a.scale_log2 == 0.f ? 1.f : fabsf(a.scale_log2);
-  while (true) {
+  // n counts this half's tiles over all units of the CTA, as the issuers do: tile n is in buffer
+  // b = n & 1, whose barriers complete for the (n >> 1)-th time
+  for (uint32_t n = 0;; ++n) {
+    const int b = static_cast<int>(n & 1u);
+    const uint32_t nph = (n >> 1) & 1u;
     if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
     const Meta mt = meta[stage];
     if (mt.flags & kDone) break;
@@ -738,14 +734,10 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       }
       pa::fence_proxy_async_smem();
     }
-    if (!pa::mbar_wait(my_s_full, s_ph)) { ok = false; break; }
-    s_ph ^= 1;
+    if (!pa::mbar_wait(&s_full[2 * half + b], nph)) { ok = false; break; }
     pa::tc_fence_after();
     float sv[kTile];
-    if (warp_active) pa::tmem_ld64(tS + lane_base, sv);
-    // S_h may be overwritten by the next tile's S from here on
-    pa::tc_fence_before();
-    pa::mbar_arrive(&s_free[half]);
+    if (warp_active) pa::tmem_ld64(tSP + 64 * b + lane_base, sv);  // waits for the load: P may replace S
     uint32_t hi[kTile / 2], lo[kTile / 2];
     float f = 1.f;
     bool rescale = false;
@@ -794,13 +786,12 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
       pa::f2_unpack(ls2[1], l2v, l3);
       l += (l0 + l1) + (l2v + l3);
     }
-    // P.V(j-1) must be complete before P is rewritten and O rescaled
-    if (pv_pending) {
-      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
-      o_ph ^= 1;
-      pv_pending = false;
+    // O is rescaled once P.V(n-1) has added to it (a warp-uniform decision; a warp with nothing to
+    // rescale does not wait)
+    if (rescale) {
+      if (!pa::mbar_wait(&o_done[2 * half + (b ^ 1)], ((n - 1) >> 1) & 1u)) { ok = false; break; }
+      pa::tc_fence_after();
     }
-    pa::tc_fence_after();
     if (warp_active) {
       if (rescale) {
 #pragma unroll 1
@@ -812,17 +803,14 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
           pa::tmem_st16(tO + lane_base + 16 * j, t);
         }
       }
-      pa::tmem_st32(tP + lane_base, hi);
-      pa::tmem_st32(tP + lane_base + 32, lo);
+      pa::tmem_st32(tSP + 64 * b + lane_base, hi);
+      pa::tmem_st32(tSP + 64 * b + lane_base + 32, lo);
       pa::tmem_wait_st();
     }
     pa::tc_fence_before();
-    pa::mbar_arrive(my_p_full);
-    pv_pending = true;
+    pa::mbar_arrive(&p_full[2 * half + b]);
     if (mt.flags & kLast) {
-      if (!pa::mbar_wait(my_o_done, o_ph)) { ok = false; break; }
-      o_ph ^= 1;
-      pv_pending = false;
+      if (!pa::mbar_wait(&o_done[2 * half + b], nph)) { ok = false; break; }
       pa::tc_fence_after();
       if (warp_active) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
