@@ -508,6 +508,33 @@ def test_prefill_mixed_batch(oracle_mod, dtype, g, d, B):
     _assert_close(out.cpu(), ref, dtype, f"prefill {dtype} g={g} d={d} B={B}")
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_prefill_many_units_per_cta(oracle_mod, dtype):
+    # about ten work units per persistent CTA, so that the tile counter, the S/P buffer parity and
+    # the barrier phases run on across units: short chunks (one 64-key tile up to several, odd and
+    # even tile counts), chunks that leave the second 128-row half without a query (at most 32
+    # tokens with g = 4) next to ones that fill both halves, and decode rows
+    g = W.generator(690)
+    S = 700
+    nq = torch.randint(2, 71, (S,), generator=g)
+    nq[::9] = 1
+    ctx = (nq + torch.randint(0, 230, (S,), generator=g)).tolist()
+    nq = nq.tolist()
+    case, q, q_start = _prefill_case(ctx, nq, 8, 2, 128, 16, dtype, 691)
+    ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                             case.scale, n_threads=0)
+    dev = case.to("cuda")
+    ws = torch.empty(api.prefill_workspace_size(case.S, case.H, 2, 128, max(ctx), max(nq)), dtype=torch.uint8,
+                     device="cuda")
+    for _ in range(2):  # twice in a row: the second call reuses the workspace the first one left
+        out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables,
+                             dev.context_lens, max_context_len=max(ctx), max_q_len=max(nq), scale=case.scale,
+                             out_dtype=torch.float32, workspace=ws)
+        torch.cuda.synchronize()
+        assert api.workspace_error(ws) == 0
+        _assert_close(out.cpu(), ref, dtype, f"prefill, many units per CTA, {dtype}")
+
+
 @pytest.fixture(params=["tcgen05", "mma_sync"])
 def prefill_consumer(request, monkeypatch):
     """pa_prefill consumers: tcgen05 with TMEM accumulators (default) or mma.sync."""
