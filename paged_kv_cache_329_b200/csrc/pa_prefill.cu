@@ -689,11 +689,24 @@ __global__ void __launch_bounds__(kUThreads, 1) prefill_umma_kernel(const __grid
   const float sl2 = a.scale_log2 == 0.f ? 1.f : fabsf(a.scale_log2);
   // n counts this half's tiles over all units of the CTA, as the issuers do: tile n is in buffer
   // b = n & 1, whose barriers complete for the (n >> 1)-th time
+  // Only a unit's first tile needs the producer's meta: the rows derive the others' position,
+  // length and last-tile flag from it, and wait for a stage's data only where they write into it
+  // (the zeroed V rows of a ragged last tile).
+  Meta mt;
+  mt.flags = kLast;  // the next tile starts a unit
   for (uint32_t n = 0;; ++n) {
     const int b = static_cast<int>(n & 1u);
     const uint32_t nph = (n >> 1) & 1u;
-    if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
-    const Meta mt = meta[stage];
+    if (mt.flags & kLast) {
+      if (!pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+      mt = meta[stage];
+    } else {
+      mt.tile_pos += kTile;
+      const int kv_end = mt.qpos0 + mt.nq;  // keys 0 .. kv_end-1 for the unit's queries
+      mt.ntok = min(kTile, kv_end - mt.tile_pos);
+      mt.flags = mt.tile_pos + kTile >= kv_end ? kLast : 0;
+      if (mt.ntok < kTile && !pa::mbar_wait(&full[stage], phase)) { ok = false; break; }
+    }
     if (mt.flags & kDone) break;
     if (mt.flags & kFirst) {
       const int tok = r / G, h = r % G;
