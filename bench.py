@@ -509,6 +509,7 @@ def run_pa(args, rank, world, local_rank):
         return None
 
     peak, peak_kind = load_peaks()
+    uniq_bytes = wl.unique_kv_bytes(traj[0]["tables"].cpu(), lens) if hasattr(wl, "unique_kv_bytes") else None
     value = aggregate_value(step_bytes, K, world, total_ms)
     achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
     ms_per_step = total_ms / K
@@ -534,16 +535,18 @@ def run_pa(args, rank, world, local_rank):
             "seq_len": f"mean {statistics.mean(lens.tolist()):.0f}, max {max(lens.tolist())}",
             "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
             "partition_size": wl.P,
-            "l2": (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step, no flush"
-                   if kv_bytes > L2_BYTES else
+            "l2": (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step"
+                   + (f" ({uniq_bytes / 1e9:.2f} GB in distinct blocks: blocks shared by several sequences are "
+                      f"read once per sequence, partly from L2)" if uniq_bytes is not None else "") + ", no flush"
+                   if (uniq_bytes if uniq_bytes is not None else kv_bytes) > L2_BYTES else
                    f"warm: the {kv_bytes / 1e6:.1f} MB of K/V read per step fit in L2 (no flush)"),
             "step": "host block manager -> pa_decode_step (COW copies, slot writes and the decode plan in one "
                     "kernel, then decode and combine)",
             "step_bytes": round(step_bytes),
             "cow_pairs_per_step": n_pairs,
             "trajectory_steps": n_traj,
-            **({"unique_kv_bytes_step0": wl.unique_kv_bytes(traj[0]["tables"].cpu(), lens),
-                "logical_kv_bytes_step0": traj[0]["kv_bytes"]} if hasattr(wl, "unique_kv_bytes") else {}),
+            **({"unique_kv_bytes_step0": uniq_bytes,
+                "logical_kv_bytes_step0": traj[0]["kv_bytes"]} if uniq_bytes is not None else {}),
         },
         "kernel_ms": {"step": round(ms_per_step, 5), "decode": round(decode_ms, 5),
                       "step_over_decode": round(ms_per_step / decode_ms, 4),
