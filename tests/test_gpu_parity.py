@@ -508,23 +508,25 @@ def test_prefill_mixed_batch(oracle_mod, dtype, g, d, B):
     _assert_close(out.cpu(), ref, dtype, f"prefill {dtype} g={g} d={d} B={B}")
 
 
-@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-def test_prefill_many_units_per_cta(oracle_mod, dtype):
+@pytest.mark.parametrize("dtype,d,g", [(torch.float16, 128, 4), (torch.bfloat16, 128, 4), (torch.bfloat16, 128, 8),
+                                       (torch.bfloat16, 64, 1), (torch.bfloat16, 64, 8)])
+def test_prefill_many_units_per_cta(oracle_mod, dtype, d, g):
     # about ten work units per persistent CTA, so that the tile counter, the S/P buffer parity and
     # the barrier phases run on across units: short chunks (one 64-key tile up to several, odd and
-    # even tile counts), chunks that leave the second 128-row half without a query (at most 32
-    # tokens with g = 4) next to ones that fill both halves, and decode rows
-    g = W.generator(690)
-    S = 700
-    nq = torch.randint(2, 71, (S,), generator=g)
+    # even tile counts), chunks that leave the second 128-row half without a query (at most 128 / g
+    # tokens) next to ones that fill both halves, and decode rows; d = 64 has one 128-byte panel and
+    # a deeper K/V ring
+    gen = W.generator(690 + g + d)
+    S = 700 if g <= 4 else 400
+    nq = torch.randint(2, 256 // g + 8, (S,), generator=gen)
     nq[::9] = 1
-    ctx = (nq + torch.randint(0, 230, (S,), generator=g)).tolist()
+    ctx = (nq + torch.randint(0, 230, (S,), generator=gen)).tolist()
     nq = nq.tolist()
-    case, q, q_start = _prefill_case(ctx, nq, 8, 2, 128, 16, dtype, 691)
+    case, q, q_start = _prefill_case(ctx, nq, 2 * g, 2, d, 16, dtype, 691)
     ref = oracle_mod.prefill(q, q_start, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
                              case.scale, n_threads=0)
     dev = case.to("cuda")
-    ws = torch.empty(api.prefill_workspace_size(case.S, case.H, 2, 128, max(ctx), max(nq)), dtype=torch.uint8,
+    ws = torch.empty(api.prefill_workspace_size(case.S, case.H, 2, d, max(ctx), max(nq)), dtype=torch.uint8,
                      device="cuda")
     for _ in range(2):  # twice in a row: the second call reuses the workspace the first one left
         out = api.pa_prefill(q.cuda(), q_start.cuda(), dev.k_cache, dev.v_cache, dev.block_tables,
@@ -532,7 +534,7 @@ def test_prefill_many_units_per_cta(oracle_mod, dtype):
                              out_dtype=torch.float32, workspace=ws)
         torch.cuda.synchronize()
         assert api.workspace_error(ws) == 0
-        _assert_close(out.cpu(), ref, dtype, f"prefill, many units per CTA, {dtype}")
+        _assert_close(out.cpu(), ref, dtype, f"prefill, many units per CTA, {dtype} d={d} g={g}")
 
 
 @pytest.fixture(params=["tcgen05", "mma_sync"])
