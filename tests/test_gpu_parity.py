@@ -356,9 +356,12 @@ def test_decode_step_without_pairs_or_tokens(oracle_mod):
 
 # ---- the captured step (pa_step_*) ------------------------------------------------------------------
 
-def test_captured_step_matches_separate_calls(oracle_mod):
+@pytest.mark.parametrize("max_pairs", [None, 9000])
+def test_captured_step_matches_separate_calls(oracle_mod, max_pairs):
     # Shared-prefix trajectory: forks create copy-on-write pairs every step.  Each replay of the
-    # graph must equal the oracle applied to the same block manager state.
+    # graph must equal the oracle applied to the same block manager state.  With room for more
+    # pairs than the fused step's prologue takes, the graph holds the copy, write and decode calls
+    # instead (the pair count still read on the device).
     B, H, Hk, d, dt = 16, 32, 8, 128, torch.bfloat16
     mgr = api.BlockManager(512, B)
     g = W.generator(400)
@@ -371,7 +374,8 @@ def test_captured_step_matches_separate_calls(oracle_mod):
         roots.append([root] + [mgr.seq_fork(root) for _ in range(3)])
     kd, vd = kc.cuda(), vc.cuda()
     S = 16
-    step = api.DecodeStep(kd, vd, S, H, 32, 512, out_dtype=torch.float32)
+    step = api.DecodeStep(kd, vd, S, H, 32, 512, out_dtype=torch.float32,
+                          **({} if max_pairs is None else {"max_pairs": max_pairs}))
     k_ref, v_ref = kc.clone(), vc.clone()
     rnd = torch.Generator().manual_seed(9)
     for it in range(3):
