@@ -399,6 +399,12 @@ def test_captured_step_matches_separate_calls(oracle_mod, max_pairs):
         ref = oracle_mod.decode(step.h_query, k_ref, v_ref, step.h_tables, step.h_lens)
         assert pairs.shape[0] > 0 or it > 0
         _assert_close(out, ref, dt, f"captured step {it}")
+    # the same graph enqueued without waiting (launch): the last step again, whose copies and writes
+    # repeat the same bytes, gives the same output once the stream has reached it
+    step.h_out.zero_()
+    step.launch(torch.cuda.current_stream())
+    torch.cuda.current_stream().synchronize()
+    _assert_close(step.h_out.clone(), ref, dt, "captured step, launch()")
     assert torch.equal(kd.cpu().view(torch.int16), k_ref.view(torch.int16))
     assert torch.equal(vd.cpu().view(torch.int16), v_ref.view(torch.int16))
     assert api.workspace_error(step.workspace) == 0
