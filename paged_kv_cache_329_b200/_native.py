@@ -65,13 +65,14 @@ SIGNATURES = {
     "pa_seq_create": (I, [P, I32P]),
     "pa_seq_fork": (I, [P, ctypes.c_int32, I32P]),
     "pa_seq_free": (I, [P, ctypes.c_int32]),
-    "pa_seq_fork_batch": (I, [P, I32P, I, I32P]),
-    "pa_seq_free_batch": (I, [P, I32P, I]),
+    # batch calls take their arrays as plain addresses (a tensor's data_ptr()): no per-call casts
+    "pa_seq_fork_batch": (I, [P, P, I, P]),
+    "pa_seq_free_batch": (I, [P, P, I]),
     "pa_seq_len": (I, [P, ctypes.c_int32]),
     "pa_seq_num_blocks": (I, [P, ctypes.c_int32]),
     "pa_seq_reserve_slots": (I, [P, ctypes.c_int32, I, I64P, I32P, IP]),
-    "pa_seq_reserve_slots_batch": (I, [P, I32P, I, I, I64P, I32P, IP, IP]),
-    "pa_build_block_tables": (I, [P, I32P, I, I32P, I, I32P]),
+    "pa_seq_reserve_slots_batch": (I, [P, P, I, I, P, P, IP, IP]),
+    "pa_build_block_tables": (I, [P, P, I, P, I, P]),
 }
 
 _lib = None

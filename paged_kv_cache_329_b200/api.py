@@ -43,6 +43,21 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _host_i32(x):
+    """An input id array as a contiguous int32 CPU tensor (converted only when it is not one)."""
+    if isinstance(x, torch.Tensor):
+        if x.device.type == "cpu" and x.dtype == torch.int32 and x.is_contiguous():
+            return x
+        return x.to(device="cpu", dtype=torch.int32).contiguous()
+    return torch.tensor(list(x), dtype=torch.int32)
+
+
+def _check_host(t, dtype, n, what):
+    """An output array the native code writes through a plain address: CPU, contiguous, dtype, size."""
+    if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous() or t.numel() < n:
+        raise ValueError(f"{what} must be a contiguous {dtype} CPU tensor of at least {n} elements")
+
+
 def _cuda(*ts):
     for t in ts:
         if not t.is_cuda or not t.is_contiguous():
@@ -348,16 +363,14 @@ class BlockManager:
 
     def seq_fork_batch(self, parents):
         """Fork each parent in order; returns the children as an int32 tensor."""
-        p = parents if isinstance(parents, torch.Tensor) else torch.tensor(list(parents), dtype=torch.int32)
+        p = _host_i32(parents)
         kids = torch.empty(p.numel(), dtype=torch.int32)
-        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
-        _check(self._lib.pa_seq_fork_batch(self._h, i32(p), p.numel(), i32(kids)))
+        _check(self._lib.pa_seq_fork_batch(self._h, p.data_ptr(), p.numel(), kids.data_ptr()))
         return kids
 
     def seq_free_batch(self, seq_ids):
-        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
-        _check(self._lib.pa_seq_free_batch(self._h, ctypes.cast(ids.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
-                                           ids.numel()))
+        ids = _host_i32(seq_ids)
+        _check(self._lib.pa_seq_free_batch(self._h, ids.data_ptr(), ids.numel()))
 
     def seq_len(self, sid: int) -> int:
         return self._lib.pa_seq_len(self._h, sid)
@@ -376,27 +389,29 @@ class BlockManager:
     def reserve_slots_batch(self, seq_ids, n_new: int = 1, slots=None, pairs=None):
         """One step for a batch: n_new slots per sequence.  Returns (slots int64 [S*n_new] tensor,
         pairs int32 [n_cow, 2] tensor).  `slots`/`pairs` may be preallocated (pinned) CPU tensors."""
-        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
+        ids = _host_i32(seq_ids)
         S = ids.numel()
         if slots is None:
             slots = torch.empty(S * n_new, dtype=torch.int64)
         if pairs is None:
             pairs = torch.empty((max(S, 1), 2), dtype=torch.int32)
+        _check_host(slots, torch.int64, S * n_new, "slots")
+        _check_host(pairs, torch.int32, 2 * max(S, 1), "pairs")
         n_cow, n_done = ctypes.c_int(0), ctypes.c_int(0)
-        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
-        i64 = ctypes.cast(slots.data_ptr(), ctypes.POINTER(ctypes.c_int64))
-        _check(self._lib.pa_seq_reserve_slots_batch(self._h, i32(ids), S, n_new, i64, i32(pairs),
-                                                    ctypes.byref(n_cow), ctypes.byref(n_done)))
+        _check(self._lib.pa_seq_reserve_slots_batch(self._h, ids.data_ptr(), S, n_new, slots.data_ptr(),
+                                                    pairs.data_ptr(), ctypes.byref(n_cow), ctypes.byref(n_done)))
         return slots, pairs[: n_cow.value]
 
     def build_block_tables(self, seq_ids, max_blocks_per_seq: int, tables=None, lens=None):
         """Returns (tables int32 [S, max_blocks] CPU tensor, context_lens int32 [S] CPU tensor)."""
-        ids = seq_ids if isinstance(seq_ids, torch.Tensor) else torch.tensor(list(seq_ids), dtype=torch.int32)
+        ids = _host_i32(seq_ids)
         S = ids.numel()
         if tables is None:
             tables = torch.empty((S, max_blocks_per_seq), dtype=torch.int32)
         if lens is None:
             lens = torch.empty((S,), dtype=torch.int32)
-        i32 = lambda t: ctypes.cast(t.data_ptr(), ctypes.POINTER(ctypes.c_int32))
-        _check(self._lib.pa_build_block_tables(self._h, i32(ids), S, i32(tables), max_blocks_per_seq, i32(lens)))
+        _check_host(tables, torch.int32, S * max_blocks_per_seq, "tables")
+        _check_host(lens, torch.int32, S, "lens")
+        _check(self._lib.pa_build_block_tables(self._h, ids.data_ptr(), S, tables.data_ptr(), max_blocks_per_seq,
+                                               lens.data_ptr()))
         return tables, lens

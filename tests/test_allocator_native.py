@@ -180,3 +180,25 @@ def test_batched_fork_and_free_equal_single_calls():
     with pytest.raises(api.PAError):
         nat.seq_free_batch([kids[0], 999])
     assert nat.seq_len(kids[0]) == -1          # freed before the unknown id stopped the batch
+
+
+def test_batch_calls_check_their_host_arrays():
+    # the batch calls hand plain addresses to the library: arrays it would write through must be
+    # contiguous CPU tensors of the right type and size, and id arrays of another type are converted
+    mgr = api.BlockManager(64, 16)
+    seqs = [mgr.seq_create() for _ in range(4)]
+    slots, pairs = mgr.reserve_slots_batch(torch.tensor(seqs, dtype=torch.int64), 3)   # ids converted
+    assert slots.shape == (12,) and pairs.shape == (0, 2)
+    with pytest.raises(ValueError):
+        mgr.reserve_slots_batch(seqs, 1, torch.empty(4, dtype=torch.int32))             # wrong slot type
+    with pytest.raises(ValueError):
+        mgr.reserve_slots_batch(seqs, 2, torch.empty(4, dtype=torch.int64))             # too small
+    with pytest.raises(ValueError):
+        mgr.build_block_tables(seqs, 4, torch.empty((4, 4), dtype=torch.int32)[:, :2])  # not contiguous
+    with pytest.raises(ValueError):
+        mgr.build_block_tables(seqs, 4, None, torch.empty(4, dtype=torch.int64))        # wrong lens type
+    tables, lens = mgr.build_block_tables(seqs, 4)
+    assert lens.tolist() == [3, 3, 3, 3] and (tables[:, 0] >= 0).all() and (tables[:, 1:] == -1).all()
+    kids = mgr.seq_fork_batch(torch.tensor(seqs, dtype=torch.int32)[::2])              # strided ids
+    assert kids.tolist() == [4, 5]
+    mgr.seq_free_batch(kids)
