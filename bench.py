@@ -246,14 +246,21 @@ def code_sha256(path):
     return hashlib.sha256("\n".join(ln for ln in lines if ln.strip()).encode()).hexdigest()
 
 
+PROFILED = {  # workload -> (ncu summary, sources its dominant kernel is built from)
+    "gqa8k_bf16": ("decode_kernel_gqa8k_bf16.md", ("pa_decode.cu", "pa_device.cuh")),
+    "prefill_mixed_bf16": ("prefill_umma_kernel_mixed_bf16.md", ("pa_prefill.cu", "pa_device.cuh")),
+}
+
+
 def profiled_traffic(args):
-    """DRAM bytes per decode launch from the committed ncu summary, if the code it was captured on
-    is the current code (comments aside) and the run is the workload it was captured on
-    (gqa8k_bf16, library-default partition and B, all sequences)."""
-    if args.workload != "gqa8k_bf16" or args.partition or args.block_size or args.seqs:
+    """DRAM bytes per launch of the workload's dominant kernel from the committed ncu summary, if
+    the code it was captured on is the current code (comments aside) and the run is the workload it
+    was captured on (library-default partition and B, all sequences)."""
+    if args.workload not in PROFILED or args.partition or args.block_size or args.seqs:
         return None
-    path = os.path.join(ROOT, "profiles", "decode_kernel_gqa8k_bf16.md")
-    srcs = [os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", f) for f in ("pa_decode.cu", "pa_device.cuh")]
+    name, files = PROFILED[args.workload]
+    path = os.path.join(ROOT, "profiles", name)
+    srcs = [os.path.join(ROOT, "paged_kv_cache_329_b200", "csrc", f) for f in files]
     try:
         text = open(path).read()
         want = dict(re.findall(r"code_sha256\((\S+)\):\s*([0-9a-f]{64})", text))
@@ -781,9 +788,13 @@ def run_prefill(args, rank, world, local_rank):
                        "flops_per_step": flops, "unique_kv_bytes": kv_bytes},
             "kv_gbs_unique": round(world * kv_bytes * args.steps / (ms * 1e-3) / 1e9, 2),
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak, "peak_kind": kind,
-                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
+                         "kernel": "pa_prefill (prefill_umma_kernel dominant), CUDA events around each of K calls",
+                         "traffic": profiled_traffic(args),
                          "peak_burst": burst, "frac_of_burst": round(tflops / world / burst, 4)},
-            "clocks": clock_info, "gpu_launches": 2 * args.steps}
+            # per call: prefill_plan_kernel and prefill_umma_kernel for the prompt chunks, then
+            # plan_kernel, decode_kernel and combine_kernel for the one-token rows
+            "clocks": clock_info, "gpu_launches": 5 * args.steps}
 
 
 def run_cache_ops(args, rank, world, local_rank):
