@@ -28,6 +28,7 @@
 //   * pa_decode_step puts a step's copy-on-write copies, slot writes and the plan into one
 //     prologue kernel ahead of the decode grid ("PagedAttention原理", "解决COW": copy, then write,
 //     then read), and pa_prefill hands its one-token sequences to these kernels (rows q_start[s]).
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -1411,18 +1412,23 @@ template <class T, int D, int G, bool kMma>
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeArgs& a, int max_units,
                           cudaStream_t st) {
   using C = Cfg<T, D, G>;
-  static int occupancy = -1;  // per instantiation; device properties are uniform on a B200 node
+  // the shared-memory attribute belongs to the current context (each device keeps its own, a device
+  // reset drops it): set again whenever the context differs from the one it was set in
+  static std::atomic<unsigned long long> ready_ctx{0};
+  static std::atomic<int> occupancy{1};
   cudaError_t e = cudaSuccess;
-  if (occupancy < 0) {
+  const unsigned long long ctx = pa::current_context_id();
+  if (ctx == 0 || ready_ctx.load(std::memory_order_acquire) != ctx) {
     e = cudaFuncSetAttribute(decode_kernel<T, D, G, kMma>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<T, D, G, kMma>, kThreads, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    occupancy = occ < 1 ? 1 : occ;
+    occupancy.store(occ < 1 ? 1 : occ, std::memory_order_relaxed);
+    ready_ctx.store(pa::current_context_id(), std::memory_order_release);
   }
   const DeviceInfo di = device_info();
-  long long grid = static_cast<long long>(di.sms) * occupancy;
+  long long grid = static_cast<long long>(di.sms) * occupancy.load(std::memory_order_relaxed);
   if (grid > max_units) grid = max_units;
   if (grid < 1) grid = 1;
   return launch_pdl(decode_kernel<T, D, G, kMma>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::kSmemBytes,
@@ -1488,6 +1494,29 @@ int max_parts_for(int max_context_len, int P) {
 }
 
 }  // namespace
+
+unsigned long long pa::current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 
 extern "C" int pa_decode_default_partition(int S, int Hk, int max_context_len) {
   return default_partition(S, Hk, max_context_len);
@@ -1773,29 +1802,6 @@ struct NoAllocSlot {
 };
 NoAllocSlot g_noalloc[kMaxDevices];
 
-// Id of the calling thread's current context (0 if it cannot be had, which forces a lookup).
-unsigned long long current_context_id() {
-  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
-    return 0;
-  return id;
-}
-
 cudaError_t noalloc_scratch(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1803,13 +1809,13 @@ cudaError_t noalloc_scratch(void** ptr) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   NoAllocSlot& slot = g_noalloc[dev];
-  const unsigned long long ctx_id = current_context_id();  // 0 before the runtime has made one current
+  const unsigned long long ctx_id = pa::current_context_id();  // 0 before the runtime has made one current
   if (!slot.ptr || ctx_id == 0 || slot.ctx_id != ctx_id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's context current if needed
     if (e != cudaSuccess) return e;
     slot.ptr = p;
-    slot.ctx_id = current_context_id();
+    slot.ctx_id = pa::current_context_id();
   }
   *ptr = slot.ptr;
   return cudaSuccess;

@@ -17,6 +17,11 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t elem_size(pa_dtype t) { return t == PA_F32 ? 4 : 2; }
 inline bool valid_dtype(int t) { return t == PA_F32 || t == PA_F16 || t == PA_BF16; }
 
+// Id of the calling thread's current CUDA context, 0 if there is none or it cannot be had.  The
+// driver never reuses an id within a process, so a set-up that belongs to a context (a kernel's
+// shared-memory size attribute, kept per device and lost with a device reset) can be keyed on it.
+unsigned long long current_context_id();
+
 // Most copy pairs pa_decode_step takes (their destinations are held in shared memory).
 constexpr int kMaxStepPairs = 8192;
 

@@ -18,6 +18,7 @@
 // 16-bit hi + lo pair, with the online softmax per row in fp32.  Causal masking compares each
 // key's position with the row's own position.  Every warp finishes its rows alone, so there is
 // no cross-warp merge; units are listed longest key range first.
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -898,19 +899,23 @@ bool cache_map(CUtensorMap* map, const void* base, pa_dtype dt, int d, long long
 template <class T, int D, int G>
 cudaError_t launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
   using C = PCfg<D>;
-  static int occupancy = -1;
-  if (occupancy < 0) {
+  // per context: the shared-memory attribute is kept per device and lost with a device reset
+  static std::atomic<unsigned long long> ready_ctx{0};
+  static std::atomic<int> occupancy{1};
+  const unsigned long long ctx = pa::current_context_id();
+  if (ctx == 0 || ready_ctx.load(std::memory_order_acquire) != ctx) {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, prefill_kernel<T, D, G>, kThreads, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    occupancy = occ < 1 ? 1 : occ;
+    occupancy.store(occ < 1 ? 1 : occ, std::memory_order_relaxed);
+    ready_ctx.store(pa::current_context_id(), std::memory_order_release);
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long long grid = static_cast<long long>(sms) * occupancy;
+  long long grid = static_cast<long long>(sms) * occupancy.load(std::memory_order_relaxed);
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
   return launch_pdl(prefill_kernel<T, D, G>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), C::kSmemBytes, st,
@@ -920,8 +925,9 @@ cudaError_t launch(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, 
 template <class T, int D, int G>
 cudaError_t launch_umma(const CUtensorMap& tk, const CUtensorMap& tv, const Args& a, long long units, cudaStream_t st) {
   using C = UCfg<D>;
-  static bool ready = false;
-  if (!ready) {
+  static std::atomic<unsigned long long> ready_ctx{0};  // per context, as in launch()
+  const unsigned long long ctx = pa::current_context_id();
+  if (ctx == 0 || ready_ctx.load(std::memory_order_acquire) != ctx) {
     cudaError_t e = cudaFuncSetAttribute(prefill_umma_kernel<T, D, G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -932,7 +938,7 @@ cudaError_t launch_umma(const CUtensorMap& tk, const CUtensorMap& tv, const Args
     if (e != cudaSuccess) return e;
     if (static_cast<long long>(fa.numRegs) * kUThreads < 2LL * 128 * (kRegsRows + kRegsOther))
       return cudaErrorInvalidConfiguration;
-    ready = true;
+    ready_ctx.store(pa::current_context_id(), std::memory_order_release);
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
