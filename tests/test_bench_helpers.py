@@ -56,3 +56,26 @@ def test_clock_sampler_windows():
     c.windows = [(10.06, 10.07)]
     out = c.finish()
     assert out["samples"] == 2 and out["reasons"] == ["sw_power_cap"] and "hw_slowdown" not in out["reasons"]
+
+
+def test_profiled_traffic_matches_the_committed_sources():
+    # the roofline's traffic comes from the committed ncu summaries only while their recorded code
+    # hashes are those of the current sources; a kernel edit without a new capture drops it to null
+    class A:
+        partition = block_size = seqs = 0
+    for wl in bench.PROFILED:
+        A.workload = wl
+        t = bench.profiled_traffic(A)
+        assert t is not None and t > 1e8, f"{wl}: the profile's code hashes do not match the sources"
+    A.workload, A.seqs = "gqa8k_bf16", 64
+    assert bench.profiled_traffic(A) is None          # another workload than the one captured
+    A.workload, A.seqs = "long_bf16", 0
+    assert bench.profiled_traffic(A) is None
+
+
+def test_code_hash_ignores_comments(tmp_path):
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text("int f() {\n  return 1;  // one\n}\n")
+    b.write_text("/* header */\nint f() {\n\n  return 1;\n}\n")
+    c.write_text("int f() {\n  return 2;\n}\n")
+    assert bench.code_sha256(str(a)) == bench.code_sha256(str(b)) != bench.code_sha256(str(c))
